@@ -1,0 +1,297 @@
+/*
+ * wqmm_oracle.c -- plain, slow CPU oracle for the anti-quant weight GEMM and
+ * its int8 sibling.  TEST INFRASTRUCTURE ONLY: it is loaded by the tests, by
+ * the package's smoke check and by the benchmark's CPU-baseline leg, never by
+ * the product path.  It shares no code, header or table with the CUDA path.
+ *
+ * What it computes (written out from the definitions, no blocking/fusion):
+ *
+ *  wqmm  -- aclnnWeightQuantMatmulAllReduce, "计算公式":
+ *           output = x1 @ ((x2 + antiquantOffset) * antiquantScale) + bias + x3
+ *           (the AllReduce is the identity for one rank).  The offset is ADDED
+ *           to the weight before the scale is applied.  Per-tensor scale has
+ *           shape (1), per-channel (n) or (1,n), per-group (ceil(k/G), n) with
+ *           row k//G used for weight row k ("约束说明", and the golden script
+ *           description of "仓库中的验证与配套资源", which expands per-group
+ *           factors with repeat_interleave(group_size, dim=0)).
+ *  qmm   -- aclnnQuantMatmulAllReduceV2, "Function", cases 1 and 2:
+ *           output = dequantScale * pertokenScale * (x1_int8 @ x2_int8 + bias_int32) + x3
+ *
+ * Arithmetic: every weight, scale, offset, activation and bias value is decoded
+ * exactly into a double; the dot product is summed in fp64 in the fixed order
+ * k = 0 .. k-1; bias and x3 are added; the result is rounded ONCE, round to
+ * nearest even, to the output format.  The exact (pre-rounding) double is also
+ * returned, since a GPU result is compared against it.
+ * The int8 path accumulates exactly in int64, adds the int32 bias and wraps to
+ * int32 (two's complement) -- the accumulator a 32-bit integer MMA produces.
+ *
+ * Format decoders/encoders are written from IEEE 754-2008 binary16, the bf16
+ * truncated-binary32 layout (1 sign, 8 exponent, 7 fraction bits) and the OCP
+ * 8-bit floating point specification (E4M3FN: bias 7, no infinities, only
+ * S.1111.111 is NaN, subnormals kept, max 448).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* dtype codes used by this file's entry points (the oracle's own numbering) */
+#define OR_F16 1
+#define OR_BF16 2
+#define OR_F32 3
+#define OR_I8 4
+#define OR_I4 5
+#define OR_FP8E4M3 7
+
+/* scale/offset modes */
+#define OR_PER_TENSOR 0
+#define OR_PER_CHANNEL 1
+#define OR_PER_GROUP 2
+
+/* ------------------------------------------------------------------ decoders */
+
+/* binary16: value = (-1)^s * 2^(e-15) * 1.f for 1 <= e <= 30,
+ *           (-1)^s * 2^-14 * 0.f for e == 0, inf/NaN for e == 31. */
+double oracle_f16_to_double(uint16_t h) {
+    int s = (h >> 15) & 1, e = (h >> 10) & 0x1F, f = h & 0x3FF;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -24); /* 0.f * 2^-14 = f * 2^-24 */
+    else if (e == 31)
+        v = f ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + f), e - 25); /* 1.f * 2^(e-15) */
+    return s ? -v : v;
+}
+
+/* bf16: the upper half of a binary32: 8-bit exponent, bias 127, 7 fraction bits. */
+double oracle_bf16_to_double(uint16_t b) {
+    int s = (b >> 15) & 1, e = (b >> 7) & 0xFF, f = b & 0x7F;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -133); /* 0.f * 2^-126 = f * 2^-133 */
+    else if (e == 255)
+        v = f ? NAN : INFINITY;
+    else
+        v = ldexp((double)(128 + f), e - 134); /* 1.f * 2^(e-127) */
+    return s ? -v : v;
+}
+
+/* OCP FP8 E4M3FN: 4-bit exponent (bias 7), 3 fraction bits, no infinities,
+ * exponent 15 with fraction 7 is NaN, subnormals 0.f * 2^-6. */
+double oracle_e4m3_to_double(uint8_t c) {
+    int s = (c >> 7) & 1, e = (c >> 3) & 0xF, f = c & 0x7;
+    double v;
+    if (e == 15 && f == 7)
+        v = NAN;
+    else if (e == 0)
+        v = ldexp((double)f, -9); /* 0.f * 2^-6 = f * 2^-9 */
+    else
+        v = ldexp((double)(8 + f), e - 10); /* 1.f * 2^(e-7) */
+    return s ? -v : v;
+}
+
+/* ------------------------------------------------------------------ encoders */
+
+/* Round x to the nearest value with `p` significant bits (implicit bit
+ * included), minimum normal exponent `emin` (subnormal spacing
+ * 2^(emin-p+1)), ties to even.  Returns the rounded value as a double (exact,
+ * since p <= 24).  Overflow is left to the caller. */
+static double round_to_precision(double x, int p, int emin) {
+    if (x == 0.0 || !isfinite(x)) return x;
+    int e2;
+    frexp(x, &e2);    /* |x| = f * 2^e2, f in [0.5, 1) */
+    int E = e2 - 1;   /* |x| in [2^E, 2^(E+1)) */
+    if (E < emin) E = emin;
+    int qexp = E - (p - 1);           /* spacing of representable values */
+    double r = ldexp(x, -qexp);       /* exact: scaling by a power of two */
+    double ri = nearbyint(r);         /* default rounding mode: nearest, ties to even */
+    return ldexp(ri, qexp);
+}
+
+/* binary16 encode, round to nearest even; |rounded| > 65504 -> inf. */
+uint16_t oracle_double_to_f16(double x) {
+    if (isnan(x)) return 0x7E00;
+    uint16_t sign = signbit(x) ? 0x8000 : 0;
+    double a = fabs(x);
+    double r = round_to_precision(a, 11, -14);
+    if (r > 65504.0) return sign | 0x7C00;
+    if (r == 0.0) return sign;
+    int e2;
+    frexp(r, &e2);
+    int E = e2 - 1;
+    if (E < -14) { /* subnormal: r = f * 2^-24 */
+        return sign | (uint16_t)ldexp(r, 24);
+    }
+    uint16_t frac = (uint16_t)(ldexp(r, 10 - E) - 1024.0);
+    return sign | (uint16_t)((E + 15) << 10) | frac;
+}
+
+/* bf16 encode, round to nearest even from the double directly (no detour
+ * through binary32, which would round twice); overflow -> inf. */
+uint16_t oracle_double_to_bf16(double x) {
+    if (isnan(x)) return 0x7FC0;
+    uint16_t sign = signbit(x) ? 0x8000 : 0;
+    double a = fabs(x);
+    double r = round_to_precision(a, 8, -126);
+    double maxv = ldexp(255.0, 120); /* (2 - 2^-7) * 2^127 */
+    if (r > maxv) return sign | 0x7F80;
+    if (r == 0.0) return sign;
+    int e2;
+    frexp(r, &e2);
+    int E = e2 - 1;
+    if (E < -126) return sign | (uint16_t)ldexp(r, 133);
+    uint16_t frac = (uint16_t)(ldexp(r, 7 - E) - 128.0);
+    return sign | (uint16_t)((E + 127) << 7) | frac;
+}
+
+static double decode_act(int dt, uint16_t v) {
+    return dt == OR_F16 ? oracle_f16_to_double(v) : oracle_bf16_to_double(v);
+}
+
+static uint16_t encode_act(int dt, double v) {
+    return dt == OR_F16 ? oracle_double_to_f16(v) : oracle_double_to_bf16(v);
+}
+
+/* --------------------------------------------------------------- weight access */
+
+/* Value of weight element (kk, nn) of x2, viewed as a (k, n) matrix whose
+ * element (kk, nn) sits at logical linear index kk*s0 + nn*s1.
+ * int4: two's-complement nibbles, two per byte, the even linear index in the
+ * low nibble ("low nibble first"). */
+double oracle_weight_at(int w_dtype, const void* x2, int64_t s0, int64_t s1, int64_t kk, int64_t nn) {
+    int64_t idx = kk * s0 + nn * s1;
+    if (w_dtype == OR_I8) return (double)((const int8_t*)x2)[idx];
+    if (w_dtype == OR_FP8E4M3) return oracle_e4m3_to_double(((const uint8_t*)x2)[idx]);
+    /* OR_I4 */
+    uint8_t byte = ((const uint8_t*)x2)[idx >> 1];
+    int nib = (idx & 1) ? (byte >> 4) : (byte & 0xF);
+    return (double)(nib >= 8 ? nib - 16 : nib);
+}
+
+/* Every selected row/col must index the problem; returns 0 when they do. */
+static int check_selection(int64_t m, int64_t n, int64_t n_rows, const int64_t* rows, int64_t n_cols,
+                           const int64_t* cols) {
+    if (rows)
+        for (int64_t i = 0; i < n_rows; ++i)
+            if (rows[i] < 0 || rows[i] >= m) return -1;
+    if (cols)
+        for (int64_t j = 0; j < n_cols; ++j)
+            if (cols[j] < 0 || cols[j] >= n) return -1;
+    return 0;
+}
+
+/* -------------------------------------------------------------------- wqmm */
+
+/*
+ * y[i][j] = sum_k x1[i][k] * W[k][j] + bias[j] + x3[i][j],
+ * W[k][j] = (x2[k][j] + off[r(k)][c(j)]) * scale[r(k)][c(j)],
+ * r(k) = k / group_size in per-group mode, else 0; c(j) = j unless per-tensor.
+ * scale/offset element (r, c) sits at r*ss0 + c*ss1 (per-tensor: index 0).
+ *
+ * rows/cols select which outputs to evaluate (NULL = all); outputs are written
+ * densely as n_rows x n_cols.  mirror != 0 rounds every W[k][j] to the
+ * activation format before the product (a diagnostic of what a
+ * dequantise-then-MMA kernel sees; never used for grading).
+ * Returns 0, or -1 on a bad argument.
+ */
+int oracle_wqmm(int64_t m, int64_t k, int64_t n, int act_dtype, const uint16_t* x1, int w_dtype,
+                const void* x2, int64_t s0, int64_t s1, int mode, int64_t group_size,
+                const uint16_t* scale, const uint16_t* offset, int64_t ss0, int64_t ss1,
+                const uint16_t* bias, const uint16_t* x3, int64_t n_rows, const int64_t* rows,
+                int64_t n_cols, const int64_t* cols, int mirror, double* y_exact, uint16_t* y_rounded) {
+    if (m < 0 || k < 0 || n < 0) return -1;
+    if (act_dtype != OR_F16 && act_dtype != OR_BF16) return -1;
+    if (w_dtype != OR_I8 && w_dtype != OR_I4 && w_dtype != OR_FP8E4M3) return -1;
+    if (mode == OR_PER_GROUP && group_size <= 0) return -1;
+    if (rows == NULL) n_rows = m;
+    if (cols == NULL) n_cols = n;
+    if (check_selection(m, n, n_rows, rows, n_cols, cols)) return -1;
+
+#pragma omp parallel
+    {
+        double* wcol = (double*)malloc(sizeof(double) * (size_t)(k > 0 ? k : 1));
+        double* xrow = (double*)malloc(sizeof(double) * (size_t)(k > 0 ? k : 1));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t jj = 0; jj < n_cols; ++jj) {
+            int64_t j = cols ? cols[jj] : jj;
+            /* decode weight column j: W[kk][j] */
+            for (int64_t kk = 0; kk < k; ++kk) {
+                int64_t r = (mode == OR_PER_GROUP) ? kk / group_size : 0;
+                int64_t c = (mode == OR_PER_TENSOR) ? 0 : j;
+                int64_t sidx = (mode == OR_PER_TENSOR) ? 0 : r * ss0 + c * ss1;
+                double s = decode_act(act_dtype, scale[sidx]);
+                double o = offset ? decode_act(act_dtype, offset[sidx]) : 0.0;
+                double w = (oracle_weight_at(w_dtype, x2, s0, s1, kk, j) + o) * s;
+                if (mirror) w = decode_act(act_dtype, encode_act(act_dtype, w));
+                wcol[kk] = w;
+            }
+            for (int64_t ii = 0; ii < n_rows; ++ii) {
+                int64_t i = rows ? rows[ii] : ii;
+                const uint16_t* xr = x1 + i * k;
+                for (int64_t kk = 0; kk < k; ++kk) xrow[kk] = decode_act(act_dtype, xr[kk]);
+                double acc = 0.0;
+                for (int64_t kk = 0; kk < k; ++kk) acc += xrow[kk] * wcol[kk];
+                if (bias) acc += decode_act(act_dtype, bias[j]);
+                if (x3) acc += decode_act(act_dtype, x3[i * n + j]);
+                y_exact[ii * n_cols + jj] = acc;
+                if (y_rounded) y_rounded[ii * n_cols + jj] = encode_act(act_dtype, acc);
+            }
+        }
+        free(wcol);
+        free(xrow);
+    }
+    return 0;
+}
+
+/* --------------------------------------------------------------------- qmm */
+
+/*
+ * acc[i][j] = wrap32( sum_k int64(x1[i][k]) * int64(x2[k][j]) + bias[j] )
+ * y[i][j]   = double(acc) * dq[j or 0] * pt[i] + x3[i][j]
+ * dq: dq_dtype OR_BF16 (uint16 bits) or OR_F32 (float), dq_numel == 1 means
+ * per-tensor.  pt NULL means 1, bias NULL means 0, x3 NULL means 0.
+ */
+int oracle_qmm(int64_t m, int64_t k, int64_t n, const int8_t* x1, const int8_t* x2, int64_t s0, int64_t s1,
+               const int32_t* bias, int dq_dtype, const void* dq, int64_t dq_numel, const float* pt,
+               int out_dtype, const uint16_t* x3, int64_t n_rows, const int64_t* rows, int64_t n_cols,
+               const int64_t* cols, int32_t* acc_out, double* y_exact, uint16_t* y_rounded) {
+    if (m < 0 || k < 0 || n < 0) return -1;
+    if (out_dtype != OR_F16 && out_dtype != OR_BF16) return -1;
+    if (dq_dtype != OR_BF16 && dq_dtype != OR_F32) return -1;
+    if (rows == NULL) n_rows = m;
+    if (cols == NULL) n_cols = n;
+    if (check_selection(m, n, n_rows, rows, n_cols, cols)) return -1;
+
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t jj = 0; jj < n_cols; ++jj) {
+        int64_t j = cols ? cols[jj] : jj;
+        int64_t d = dq_numel == 1 ? 0 : j;
+        double dqv = dq_dtype == OR_BF16 ? oracle_bf16_to_double(((const uint16_t*)dq)[d])
+                                         : (double)((const float*)dq)[d];
+        for (int64_t ii = 0; ii < n_rows; ++ii) {
+            int64_t i = rows ? rows[ii] : ii;
+            int64_t acc = 0;
+            for (int64_t kk = 0; kk < k; ++kk)
+                acc += (int64_t)x1[i * k + kk] * (int64_t)x2[kk * s0 + j * s1];
+            if (bias) acc += bias[j];
+            int32_t a32 = (int32_t)(uint32_t)((uint64_t)acc & 0xFFFFFFFFu);
+            double y = (double)a32 * dqv * (pt ? (double)pt[i] : 1.0);
+            if (x3) y += decode_act(out_dtype, x3[i * n + j]);
+            if (acc_out) acc_out[ii * n_cols + jj] = a32;
+            if (y_exact) y_exact[ii * n_cols + jj] = y;
+            if (y_rounded) y_rounded[ii * n_cols + jj] = encode_act(out_dtype, y);
+        }
+    }
+    return 0;
+}
+
+/* Number of OpenMP threads the oracle runs with (1 when built without OpenMP). */
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
