@@ -1,0 +1,292 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.
+
+Tolerance (stated by the task for this operator): max|gpu - oracle| / max|oracle|
+<= 4e-3 for bf16 outputs and <= 1e-3 for fp16 outputs, where `oracle` is the
+exact (fp64, pre-rounding) result; the raw int32 accumulator of the int8 path
+is compared bit for bit.  Small cases span several tiles plus ragged tails in
+m, n and k and cover every mode, weight type, activation type and layout;
+full-size workloads are checked on sampled outputs the oracle evaluates one by
+one.
+"""
+import zlib
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import oracle
+import workloads as WL
+import weight_quantized_gemm_anti_b200 as W
+from weight_quantized_gemm_anti_b200 import cases as C
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"bf16": 4e-3, "f16": 1e-3}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    W.build()
+    torch.cuda.init()
+    yield
+
+
+def dec(bits: np.ndarray, act: str) -> np.ndarray:
+    bits = np.asarray(bits, dtype=np.uint16)
+    if act == "f16":
+        return bits.view(np.float16).astype(np.float64)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def gpu_bits(t) -> np.ndarray:
+    return t.view(torch.int16).cpu().numpy().view(np.uint16).reshape(-1, t.shape[-1])
+
+
+def no_device_error():
+    st, code = W.wqmm_device_error(reset=True)
+    assert st == W.SUCCESS and code == 0, f"device error word {code}"
+
+
+def rel_err(got, exact):
+    denom = np.abs(exact).max()
+    return np.abs(got - exact).max() / (denom if denom > 0 else 1.0)
+
+
+def run_wqmm(case, pack=True):
+    d = C.wqmm_to_device(case, pack=pack)
+    C.wqmm_call(d)
+    torch.cuda.synchronize()
+    no_device_error()
+    return gpu_bits(d.out)
+
+
+def check_wqmm(case, pack=True, rows=None, cols=None):
+    got = run_wqmm(case, pack=pack)
+    ye, _ = oracle.wqmm(case, rows=rows, cols=cols)
+    if rows is not None:
+        got = got[rows]
+    if cols is not None:
+        got = got[:, cols]
+    g = dec(got, case.act)
+    assert np.isfinite(g).all()
+    err = rel_err(g, ye)
+    assert err <= TOL[case.act], f"{case.name}: rel err {err:.3e}"
+    return err
+
+
+# ---------------------------------------------------------------- small cases
+SMALL = [
+    # name, x1_shape, n, act, wdt, mode, G, extras
+    ("i8_chan_f16_m16", (16, 256), 128, "f16", "i8", "channel", 0, {}),
+    ("i8_chan_bf16_ragged", (37, 96), 192, "bf16", "i8", "channel", 0, {}),
+    ("i8_tensor_bf16_m200", (200, 320), 160, "bf16", "i8", "tensor", 0, {"scale_const": 0.01, "offset_const": 3.0}),
+    ("i8_group32_bf16", (100, 192), 224, "bf16", "i8", "group", 32, {}),
+    ("i8_group96_f16", (70, 288), 96, "f16", "i8", "group", 96, {}),
+    ("i4_group128_bf16_m300", (300, 512), 320, "bf16", "i4", "group", 128, {"scale_range": (0.005, 0.05),
+                                                                           "offset_range": (-4, 4)}),
+    ("i4_group64_f16", (33, 256), 384, "f16", "i4", "group", 64, {}),
+    ("i4_chan_bf16_m1", (1, 640), 256, "bf16", "i4", "channel", 0, {}),
+    ("i4_tensor_f16", (129, 128), 128, "f16", "i4", "tensor", 0, {}),
+    ("fp8_chan_bf16", (50, 256), 192, "bf16", "fp8", "channel", 0, {"offset": False}),
+    ("fp8_chan_f16", (17, 128), 128, "f16", "fp8", "channel", 0, {"offset": False}),
+    ("i8_chan_bf16_no_offset", (64, 128), 128, "bf16", "i8", "channel", 0, {"offset": False}),
+    ("i8_chan_bf16_fractional", (40, 192), 128, "bf16", "i8", "channel", 0, {"fractional_offset": True}),
+    ("i4_group64_bf16_fractional", (24, 256), 128, "bf16", "i4", "group", 64, {"fractional_offset": True}),
+    ("i4_group64_f16_fractional", (24, 256), 128, "f16", "i4", "group", 64, {"fractional_offset": True}),
+    ("i8_group32_f16_fractional", (24, 128), 64, "f16", "i8", "group", 32, {"fractional_offset": True}),
+    ("i8_chan_bf16_big_offset", (20, 128), 96, "bf16", "i8", "channel", 0, {"offset_range": (113, 127)}),
+    ("i4_3d_bf16", (2, 9, 256), 128, "bf16", "i4", "group", 64, {}),
+    ("i8_chan_bf16_scale2d", (20, 64), 96, "bf16", "i8", "channel", 0, {"scale_2d": True}),
+    ("i8_nobias_nox3", (48, 128), 128, "bf16", "i8", "channel", 0, {"bias": False, "x3": False}),
+    ("i4_splitk_m16", (16, 4096), 256, "bf16", "i4", "group", 128, {}),
+    ("i8_splitk_m5", (5, 2048), 128, "f16", "i8", "channel", 0, {}),
+    ("i4_m64_bn64", (64, 512), 256, "bf16", "i4", "group", 64, {}),
+    ("i4_m20_bn32", (20, 512), 512, "bf16", "i4", "group", 32, {}),
+]
+
+
+@pytest.mark.parametrize("spec", SMALL, ids=[s[0] for s in SMALL])
+def test_wqmm_small_parity(spec):
+    name, x1s, n, act, wdt, mode, G, extra = spec
+    case = WL.make_wqmm_case(name=name, x1_shape=x1s, n=n, act=act, wdt=wdt, mode=mode, group_size=G,
+                             seed=zlib.crc32(name.encode()) % 10000, **extra)
+    check_wqmm(case)
+
+
+@pytest.mark.parametrize("wdt,mode,G", [("i8", "group", 32), ("i4", "group", 64), ("fp8", "channel", 0),
+                                        ("i8", "channel", 0)])
+def test_wqmm_transposed_weight(wdt, mode, G):
+    case = WL.make_wqmm_case(name="t", x1_shape=(40, 256), n=192 if wdt != "i4" else 256, act="bf16", wdt=wdt,
+                             mode=mode, group_size=G, x2_transposed=True, scale_transposed=(mode == "group"),
+                             offset=(wdt != "fp8"), seed=7)
+    check_wqmm(case, pack=True)
+    check_wqmm(case, pack=False)
+
+
+def test_nd_weight_packed_inside_run_matches_prepacked():
+    case = WL.make_wqmm_case(x1_shape=(77, 256), n=192, act="bf16", wdt="i8", mode="group", group_size=64, seed=3)
+    a = run_wqmm(case, pack=True)
+    b = run_wqmm(case, pack=False)
+    assert np.array_equal(a, b)
+
+
+def test_empty_k_gives_bias_plus_x3():
+    case = WL.make_wqmm_case(x1_shape=(10, 0), n=96, act="bf16", wdt="i8", mode="channel", seed=4)
+    got = run_wqmm(case, pack=False)
+    _, yr = oracle.wqmm(case)
+    assert np.array_equal(got, yr)  # a single rounding of bias + x3 on both sides
+
+
+def test_page_sample_all_ones_gives_130():
+    case = WL.make_wqmm_case(x1_shape=(32, 64), n=128, act="f16", wdt="i8", mode="channel", seed=0)
+    one = WL.f16_bits(np.ones(1))[0]
+    for a in (case.x1, case.scale, case.offset, case.bias, case.x3):
+        a[:] = one
+    case.x2[:] = 1
+    got = dec(run_wqmm(case, pack=False), "f16")
+    assert (got == 130.0).all()
+
+
+def test_repeated_runs_are_bitwise_deterministic():
+    case = WL.make_wqmm_case(x1_shape=(16, 4096), n=256, act="bf16", wdt="i4", mode="group", group_size=128, seed=8)
+    d = C.wqmm_to_device(case)
+    outs = []
+    for _ in range(3):
+        C.wqmm_call(d)
+        torch.cuda.synchronize()
+        outs.append(gpu_bits(d.out).copy())
+    no_device_error()
+    assert all(np.array_equal(outs[0], o) for o in outs[1:])
+
+
+# ---------------------------------------------------------------- pack kernel layout
+def _np_pack_wq_int4(q: np.ndarray) -> np.ndarray:
+    """Independent numpy statement of the anti-quant GEMM's int4 tile layout."""
+    k, n = q.shape
+    NB, KT = -(-n // 128), -(-k // 64)
+    u = np.zeros((NB * 128, KT * 64), dtype=np.uint32)
+    u[:n, :k] = (q.T.astype(np.int64) + 8) & 0xF
+    u[n:, :] = 8
+    u[:, k:] = 8
+    out = np.zeros((NB, KT, 2, 128, 4), dtype=np.uint32)
+    for c in range(2):
+        for w in range(4):
+            word = np.zeros((NB * 128, KT), dtype=np.uint32)
+            for j in range(4):
+                word |= u[:, c * 32 + 8 * w + 2 * j::64][:, :KT] << (4 * j)
+                word |= u[:, c * 32 + 8 * w + 2 * j + 1::64][:, :KT] << (16 + 4 * j)
+            out[:, :, c, :, w] = word.reshape(NB, 128, KT).transpose(0, 2, 1)
+    return out.reshape(-1).view(np.uint8)
+
+
+def test_pack_kernel_int4_layout():
+    case = WL.make_wqmm_case(x1_shape=(1, 128), n=192, act="bf16", wdt="i4", mode="channel", seed=5)
+    d = C.wqmm_to_device(case, pack=True)
+    torch.cuda.synchronize()
+    got = d.packed.cpu().numpy()
+    lo, hi = case.x2 & 0xF, case.x2 >> 4
+    q = np.empty((128, 192), dtype=np.int64)
+    q[:, 0::2], q[:, 1::2] = lo, hi
+    q = np.where(q >= 8, q - 16, q)
+    assert np.array_equal(got, _np_pack_wq_int4(q))
+
+
+def test_pack_kernel_int8_qmm_layout():
+    case = WL.make_qmm_case(x1_shape=(4, 256), n=320, seed=6)
+    d = C.qmm_to_device(case, pack=True)
+    torch.cuda.synchronize()
+    got = d.packed.cpu().numpy().reshape(-1)
+    k, n = 256, 320
+    NB, KT = 2, 2
+    full = np.zeros((NB * 256, KT * 128), dtype=np.uint8)
+    full[:n, :k] = case.x2.T.view(np.uint8)
+    want = np.zeros((NB, KT, 256, 8, 16), dtype=np.uint8)
+    for r in range(256):
+        for c in range(8):
+            want[:, :, r, c ^ (r & 7), :] = full.reshape(NB, 256, KT, 8, 16)[:, r, :, c, :]
+    assert np.array_equal(got, want.reshape(-1))
+
+
+# ---------------------------------------------------------------- int8 path
+QSMALL = [
+    ("q_bf16_pertoken", (32, 64), 128, "bf16", {}),
+    ("q_f16_pertoken", (32, 64), 128, "f16", {}),
+    ("q_bf16_ragged", (200, 160), 288, "bf16", {}),
+    ("q_f16_no_pertoken", (129, 256), 256, "f16", {"pertoken": False}),
+    ("q_bf16_tensor_dq", (3, 4, 96), 64, "bf16", {"dq_per_tensor": True}),
+    ("q_bf16_no_bias_x3", (64, 128), 512, "bf16", {"bias": False, "x3": False}),
+    ("q_f16_dq2d", (16, 64), 32, "f16", {"dq_2d": True}),
+]
+
+
+@pytest.mark.parametrize("spec", QSMALL, ids=[s[0] for s in QSMALL])
+def test_qmm_small_parity_and_exact_accumulator(spec):
+    name, x1s, n, out, extra = spec
+    case = WL.make_qmm_case(name=name, x1_shape=x1s, n=n, out=out, seed=zlib.crc32(name.encode()) % 1000, **extra)
+    d = C.qmm_to_device(case)
+    acc = torch.empty((case.m, n), dtype=torch.int32, device="cuda")
+    C.qmm_call(d, raw_acc=acc)
+    torch.cuda.synchronize()
+    no_device_error()
+    a_ref, ye, _ = oracle.qmm(case)
+    assert np.array_equal(acc.cpu().numpy(), a_ref)
+    g = dec(gpu_bits(d.out), out)
+    assert rel_err(g, ye) <= TOL[out]
+
+
+def test_qmm_transposed_weight_and_unpacked():
+    case = WL.make_qmm_case(x1_shape=(40, 128), n=96, x2_transposed=True, seed=12)
+    d = C.qmm_to_device(case, pack=False)
+    acc = torch.empty((case.m, case.n), dtype=torch.int32, device="cuda")
+    C.qmm_call(d, raw_acc=acc)
+    torch.cuda.synchronize()
+    a_ref, ye, _ = oracle.qmm(case)
+    assert np.array_equal(acc.cpu().numpy(), a_ref)
+    assert rel_err(dec(gpu_bits(d.out), "bf16"), ye) <= 4e-3
+
+
+def test_qmm_page_sample_all_ones_gives_66():
+    case = WL.make_qmm_case(x1_shape=(32, 64), n=128, out="f16", seed=0)
+    case.x1[:] = 1
+    case.x2[:] = 1
+    case.bias[:] = 1
+    case.dequant_scale[:] = 1.0
+    case.pertoken_scale[:] = 1.0
+    case.x3[:] = WL.f16_bits(np.ones(1))[0]
+    d = C.qmm_to_device(case)
+    C.qmm_call(d)
+    torch.cuda.synchronize()
+    assert (dec(gpu_bits(d.out), "f16") == 66.0).all()
+
+
+# ---------------------------------------------------------------- full-size workloads (sampled)
+def _sample(m, n, nr, nc, seed):
+    rng = np.random.default_rng(seed)
+    rows = np.unique(np.concatenate([[0, m - 1], rng.choice(m, size=min(nr, m), replace=False)]))
+    cols = np.unique(np.concatenate([[0, n - 1], rng.choice(n, size=min(nc, n), replace=False)]))
+    return rows, cols
+
+
+@pytest.mark.parametrize("name", WL.WORKLOAD_NAMES[:4])
+def test_full_size_workload_sampled(name):
+    case = WL.workload(name)
+    rows, cols = _sample(case.m, case.n, 96, 768, 1)
+    check_wqmm(case, rows=rows, cols=cols)
+
+
+def test_full_size_int8_workload_sampled():
+    case = WL.workload(WL.WORKLOAD_NAMES[4])
+    d = C.qmm_to_device(case)
+    acc = torch.empty((case.m, case.n), dtype=torch.int32, device="cuda")
+    C.qmm_call(d, raw_acc=acc)
+    torch.cuda.synchronize()
+    no_device_error()
+    rows, cols = _sample(case.m, case.n, 64, 512, 2)
+    a_ref, ye, _ = oracle.qmm(case, rows=rows, cols=cols)
+    assert np.array_equal(acc.cpu().numpy()[np.ix_(rows, cols)], a_ref)
+    g = dec(gpu_bits(d.out)[np.ix_(rows, cols)], "bf16")
+    assert rel_err(g, ye) <= 4e-3

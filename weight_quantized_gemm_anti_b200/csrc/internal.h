@@ -1,0 +1,102 @@
+// internal.h -- kernel parameter blocks and launchers shared by the host API
+// (api.cu) and the kernel translation units.  Not part of the public ABI.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace wqmm {
+
+// Weight kinds of the anti-quant GEMM.
+enum WeightKind : int { kW4 = 0, kW8 = 1, kWFp8 = 2 };
+// Scale / offset modes ("计算公式" symbol table: per-tensor, per-channel, per-group).
+enum QuantMode : int { kPerTensor = 0, kPerChannel = 1, kPerGroup = 2 };
+
+// Packed weight geometry for the anti-quant GEMM: tiles of 128 n-rows x 64 k,
+// tile (nb, kt) at byte ((nb * KT + kt) * tile_bytes); inside a tile, 16-byte
+// chunk c of row r sits at ((c * 128 + r) * 16).
+constexpr int kWqNBlock = 128;
+constexpr int kWqKTile = 64;
+__host__ __device__ constexpr int wq_tile_bytes(int wk) { return wk == kW4 ? 4096 : 8192; }
+// Packed weight geometry for the int8 GEMM: tiles of 256 n-rows x 128 k bytes,
+// 32 KB each, stored in the 128-byte-swizzled K-major order (16-byte chunk c of
+// row r at r * 128 + ((c ^ (r & 7)) * 16)).
+constexpr int kQNBlock = 256;
+constexpr int kQKTile = 128;
+constexpr int kQTileBytes = kQNBlock * kQKTile;
+
+struct WqParams {
+  const uint8_t* wpack;   // packed weight (see above)
+  const uint16_t* scale;  // raw f16/bf16 bits, (rows, n) row-major after any transpose
+  const uint16_t* offset; // may be null
+  const uint16_t* bias;   // may be null
+  const uint16_t* x3;     // may be null, (m, n)
+  uint16_t* out;          // (m, n)
+  float* partial;         // split-K partials [splits][m][n], or null when splits == 1
+  uint32_t* err;          // device error word
+  int64_t m;
+  int n, k;
+  int kt_total;           // ceil(k / 64)
+  int num_nb;             // ceil(n / 128)
+  int num_mb;             // ceil(m / BN)
+  int splits;             // k splits
+  int mode;               // QuantMode
+  int group_size;         // per-group only
+  int num_groups;         // rows of scale/offset in per-group mode
+};
+
+struct QParams {
+  const uint8_t* wpack;        // packed int8 weight (int8 tiling)
+  const int32_t* bias;         // may be null
+  const void* dq;              // dequant scale: bf16 bits or f32
+  const float* pertoken;       // may be null
+  const uint16_t* x3;          // may be null
+  uint16_t* out;
+  int32_t* raw_acc;            // test-only raw accumulator output, may be null
+  uint32_t* err;
+  int64_t m;
+  int n, k;
+  int kt_total;                // ceil(k / 128)
+  int num_nb;                  // ceil(n / 256)
+  int num_mb;                  // ceil(m / 128)
+  int dq_bf16;                 // 1: bf16 dequant scale, 0: f32
+  int dq_per_tensor;           // 1: dq has one element
+  int out_bf16;                // 1: bf16 output, 0: f16
+};
+
+struct PackParams {
+  const uint8_t* src;     // x2 storage
+  uint8_t* dst;           // packed output
+  int64_t s0, s1;         // logical element strides of x2 viewed as (k, n)
+  int k, n;
+  int wk;                 // WeightKind (the int8 GEMM tiling uses kW8)
+  int for_qmm;            // 1: int8-GEMM tiling
+};
+
+struct EpiParams {        // split-K reduction + epilogue, and the k == 0 case
+  const float* partial;   // [splits][m][n] (ignored when splits == 0)
+  const uint16_t* scale;
+  const uint16_t* offset;
+  const uint16_t* bias;
+  const uint16_t* x3;
+  uint16_t* out;
+  int64_t m;
+  int n;
+  int splits;
+  int mode;
+  int wk;
+  int act_bf16;
+};
+
+// Launchers (return cudaSuccess or the launch error).
+cudaError_t launch_pack(const PackParams& p, cudaStream_t s);
+cudaError_t launch_transpose_u16(const uint16_t* src, uint16_t* dst, int rows, int cols, cudaStream_t s);
+cudaError_t launch_wqmm_gemm(const CUtensorMap& tmap_x1, const WqParams& p, int bn, int wk, bool act_bf16,
+                             cudaStream_t s);
+cudaError_t launch_wqmm_epilogue(const EpiParams& p, cudaStream_t s);
+cudaError_t launch_qmm_gemm(const CUtensorMap& tmap_x1, const QParams& p, cudaStream_t s);
+
+// Device error word of the library (first kernel error code, 0 if none).
+uint32_t* device_error_word();
+
+}  // namespace wqmm
