@@ -1,0 +1,431 @@
+"""Benchmark of the anti-quant weight GEMM (W4A16, per-group g=128, m=k=n=4096) on B200.
+
+One step = phase 1 (host: validate + plan) and phase 2 (the GEMM kernel) of
+wqmm_get_workspace_size / wqmm_run on one batch of synthetic, seeded input,
+with the weight pre-packed (the packing is weight preparation, done once).
+
+  value     : TFLOP/s (2*m*n*k / device time), inputs resident in HBM, L2
+              flushed before every timed step (a 512 MB write, outside the
+              timed interval), CUDA events on the launching stream, max over ranks.
+  e2e       : the same metric through the same C-ABI calls with HOST buffers:
+              every step copies its inputs from pinned host memory and reads
+              the output back, all inside the timed interval.
+  roofline  : the GEMM kernel against the measured dense bf16 peak.
+  cpu_baseline / --impl reference : the CPU oracle timed on a bounded sample.
+
+N > 1 (torchrun): N independent replicas (one problem per GPU, no collective on
+the data path), weak scaling; value = all ranks' FLOPs / max rank time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+HEADLINE = "w4a16_g128_bf16_4096x4096x4096"
+METRIC = "anti-quant GEMM TFLOP/s & % of roofline (W4A16 g128, m=k=n=4096), 1 B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["weight_quantized_gemm_anti_b200/csrc/kernels_wqmm.cu",
+                  "weight_quantized_gemm_anti_b200/csrc/ptx.cuh",
+                  "weight_quantized_gemm_anti_b200/csrc/kernels_qmm.cu",
+                  "weight_quantized_gemm_anti_b200/csrc/kernels_aux.cu"]
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def load_traffic(workload: str):
+    """DRAM bytes per launch from a committed ncu summary, only if it was taken
+    on the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    def __init__(self):
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self, gpu_index: int):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9 or not parts[0].isdigit() or int(parts[0]) != gpu_index:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = max(mx, float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ GPU arm
+class Problem:
+    """One workload resident on the device, with prebuilt ABI descriptors."""
+
+    def __init__(self, name, device):
+        import torch
+        import workloads as WL
+        import weight_quantized_gemm_anti_b200 as W
+        from weight_quantized_gemm_anti_b200 import cases as C
+
+        self.W, self.C, self.torch = W, C, torch
+        self.name = name
+        self.case = WL.workload(name)
+        self.int8 = not hasattr(self.case, "wdt")
+        if self.int8:
+            self.dev = C.qmm_to_device(self.case, device=device)
+        else:
+            self.dev = C.wqmm_to_device(self.case, device=device)
+        torch.cuda.synchronize()
+        c = self.case
+        self.flops = 2.0 * c.m * c.n * c.k
+        self.bytes = self._algorithmic_bytes()
+        d = self.dev
+        D = W.desc
+        if self.int8:
+            self.descs = (D(d.x1), d.x2_desc, None if d.bias is None else D(d.bias),
+                          None if d.x3 is None else D(d.x3), d.dq_desc, None if d.pt is None else D(d.pt),
+                          None, "sum", 0, 1, D(d.out))
+        else:
+            self.descs = (D(d.x1), d.x2_desc, None if d.bias is None else D(d.bias), d.scale_desc, d.offset_desc,
+                          None if d.x3 is None else D(d.x3), None, "sum", 0, 1, d.group_size, D(d.out))
+        st, ws, ex = self.phase1()
+        W.wqmm_executor_destroy(ex)
+        self.ws_size = ws
+        self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
+
+    def _algorithmic_bytes(self):
+        """Each input read once plus the output written once (int4 = 0.5 B)."""
+        c = self.case
+        if self.int8:
+            b = c.m * c.k + c.k * c.n + c.m * c.n * 2
+            b += 0 if c.bias is None else 4 * c.n
+            b += c.dequant_scale.nbytes + (0 if c.pertoken_scale is None else 4 * c.m)
+            b += 0 if c.x3 is None else 2 * c.m * c.n
+            return b
+        wbytes = {"i4": 0.5, "i8": 1.0, "fp8": 1.0}[c.wdt]
+        b = c.m * c.k * 2 + c.k * c.n * wbytes + c.m * c.n * 2
+        b += c.scale.nbytes + (0 if c.offset is None else c.offset.nbytes)
+        b += 0 if c.bias is None else 2 * c.n
+        b += 0 if c.x3 is None else 2 * c.m * c.n
+        return b
+
+    def phase1(self):
+        if self.int8:
+            return self.W.qmm_get_workspace_size(*self.descs)
+        return self.W.wqmm_get_workspace_size(*self.descs)
+
+    def phase2(self, ex, stream):
+        if self.int8:
+            return self.W.qmm_run(self.ws.data_ptr(), self.ws_size, ex, stream)
+        return self.W.wqmm_run(self.ws.data_ptr(), self.ws_size, ex, stream)
+
+    def launches_per_step(self):
+        if self.int8:
+            return 1
+        c = self.case
+        # mirror of the library's split-K choice, read back from a planned executor
+        return 1 + (1 if self.ws_size > 0 else 0)
+
+
+def time_device(prob: Problem, steps: int, warmup: int, flush_bytes: int):
+    """Per-step device time of phase 1 + phase 2 (events on the launching stream,
+    L2 flushed before each step outside the timed interval)."""
+    torch = prob.torch
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(flush_bytes, dtype=torch.uint8, device=prob.ws.device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    host_p1 = 0.0
+    for i in range(warmup + steps):
+        flush.fill_(i & 0xFF)  # > L2: evicts the previous step's inputs and outputs
+        t0 = time.perf_counter()
+        st, ws, ex = prob.phase1()
+        host_p1 += time.perf_counter() - t0 if i >= warmup else 0.0
+        prob.W.check(st)
+        if i >= warmup:
+            evs[i - warmup][0].record(stream)
+        prob.W.check(prob.phase2(ex, stream))
+        if i >= warmup:
+            evs[i - warmup][1].record(stream)
+    torch.cuda.synchronize()
+    times = [a.elapsed_time(b) for a, b in evs]
+    return times, host_p1 / max(steps, 1)
+
+
+def time_e2e(prob: Problem, steps: int, warmup: int):
+    """The same calls with host buffers: H2D of every input from pinned memory,
+    phase 1 + phase 2, D2H of the output, inside one timed interval per step."""
+    torch = prob.torch
+    d = prob.dev
+    stream = torch.cuda.current_stream()
+    if prob.int8:
+        dev_inputs = [d.x1, d.packed, d.bias, d.dq, d.pt, d.x3]
+    else:
+        dev_inputs = [d.x1, d.packed, d.scale, d.offset, d.bias, d.x3]
+    pairs = []
+    for t in dev_inputs:
+        if t is None:
+            continue
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t if t.is_contiguous() else t.contiguous())
+        pairs.append((h, t))
+    out_h = torch.empty(d.out.shape, dtype=d.out.dtype, pin_memory=True)
+    h2d = sum(h.numel() * h.element_size() for h, _ in pairs)
+    d2h = out_h.numel() * out_h.element_size()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    total = 0.0
+    for i in range(warmup + steps):
+        start.record(stream)
+        for h, t in pairs:
+            if t.is_contiguous():
+                t.copy_(h, non_blocking=True)
+            else:
+                t.copy_(h.to(t.device, non_blocking=True))
+        st, ws, ex = prob.phase1()
+        prob.W.check(st)
+        prob.W.check(prob.phase2(ex, stream))
+        out_h.copy_(d.out, non_blocking=True)
+        end.record(stream)
+        end.synchronize()
+        if i >= warmup:
+            total += start.elapsed_time(end)
+    return total / steps, h2d, d2h
+
+
+def cpu_baseline(name: str, rows: int):
+    """The oracle as it stands on the host cores, on `rows` output rows of the workload."""
+    import numpy as np
+    import oracle
+    import workloads as WL
+
+    case = WL.workload(name)
+    r = np.arange(0, case.m, max(1, case.m // rows))[:rows]
+    oracle.build()
+    t0 = time.perf_counter()
+    if hasattr(case, "wdt"):
+        oracle.wqmm(case, rows=r)
+    else:
+        oracle.qmm(case, rows=r)
+    dt = time.perf_counter() - t0
+    flops = 2.0 * len(r) * case.n * case.k
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{len(r)} of {case.m} output rows x all {case.n} columns of {name} ({dt:.1f} s)"}
+
+
+def gpu_arm(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+
+    import weight_quantized_gemm_anti_b200 as W
+    W.build()
+    peaks, peak_src = load_peaks()
+    prob = Problem(args.config, f"cuda:{local}")
+    flush_bytes = 512 << 20
+
+    sampler = ClockSampler()
+    if rank == 0:
+        sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    times, host_p1 = time_device(prob, args.steps, args.warmup, flush_bytes)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop(local) if rank == 0 else None
+    total_ms = sum(times)
+    t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    st, code = W.wqmm_device_error(reset=True)
+    if st != 0 or code != 0:
+        raise RuntimeError(f"device error word {code}")
+
+    e2e_ms, h2d, d2h = time_e2e(prob, max(3, min(args.steps, 20)), 2)
+    e2e_t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+
+    extra = {}
+    if rank == 0 and world == 1 and not args.no_extra:
+        import workloads as WL
+        for nm in WL.WORKLOAD_NAMES:
+            if nm == args.config:
+                continue
+            p2 = Problem(nm, f"cuda:{local}")
+            tt, _ = time_device(p2, args.extra_steps, 3, flush_bytes)
+            ms = sum(tt) / len(tt)
+            bound_tensor = not (p2.case.m <= 64)
+            ent = {"ms_per_step": ms, "tflops": p2.flops / (ms * 1e-3) / 1e12,
+                   "gbs": p2.bytes / (ms * 1e-3) / 1e9}
+            if bound_tensor:
+                peak = peaks["bf16_tflops"] * (2.0 if p2.int8 else 1.0)
+                ent["roofline"] = {"bound": "tensor", "peak": peak, "unit": "TFLOP/s",
+                                   "frac": ent["tflops"] / peak,
+                                   "note": "int8 peak = 2 x measured bf16 (nominal ratio)" if p2.int8 else ""}
+            else:
+                ent["roofline"] = {"bound": "hbm", "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                   "frac": ent["gbs"] / peaks["hbm_gbs"]}
+            extra[nm] = ent
+            del p2
+            torch.cuda.empty_cache()
+
+    if rank == 0:
+        ms_step = max_ms / args.steps
+        flops_all = prob.flops * world * args.steps
+        value = flops_all / (max_ms * 1e-3) / 1e12
+        achieved = prob.flops / (ms_step * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"]
+        traffic = load_traffic(args.config)
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; shapes/distributions of the workload)",
+            "config": {"workload": args.config, "m": prob.case.m, "k": prob.case.k, "n": prob.case.n,
+                       "weight": "int4 packed, per-group g=128 scale+offset", "l2": "flushed before every step "
+                       "(512 MB write outside the timed interval)", "parallelism": f"replicas x{world}"},
+            "e2e": {"value": round(prob.flops * world / (float(e2e_t.item()) * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": prob.launches_per_step() * args.steps,
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic,
+                         "peak_source": f"{peak_src} bf16 burst"},
+            "clocks": clocks,
+            "host_phase1_us": round(host_p1 * 1e6, 1),
+        }
+        if extra:
+            line["configs_measured"] = extra
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(args.config, args.cpu_rows)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def reference_arm(args):
+    """The CPU oracle timed as the reference arm on the same workload and metric."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    import workloads as WL
+
+    case = WL.workload(args.config)
+    oracle.build()
+    rows_per_step = args.ref_rows
+    rng = np.random.default_rng(0)
+    total, flops = 0.0, 0.0
+    for i in range(args.warmup + args.steps):
+        r = np.sort(rng.choice(case.m, size=rows_per_step, replace=False))
+        t0 = time.perf_counter()
+        oracle.wqmm(case, rows=r) if hasattr(case, "wdt") else oracle.qmm(case, rows=r)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            total += dt
+            flops += 2.0 * rows_per_step * case.n * case.k
+    value = flops / total / 1e12
+    sample = f"{rows_per_step} random output rows x all {case.n} columns of {args.config} per step"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)", "config": {"workload": args.config, "m": case.m, "k": case.k, "n": case.n},
+            "cpu_baseline": {"kind": "oracle", "cores": oracle.num_threads(), "sample": sample, "value": value,
+                             "unit": "TFLOP/s"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="wqmm", choices=["wqmm", "reference"])
+    ap.add_argument("--config", default=HEADLINE)
+    ap.add_argument("--extra-steps", type=int, default=100)
+    ap.add_argument("--no-extra", action="store_true", help="skip the other four workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=1024)
+    ap.add_argument("--ref-rows", type=int, default=8)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        reference_arm(args)
+    else:
+        gpu_arm(args)
+
+
+if __name__ == "__main__":
+    main()

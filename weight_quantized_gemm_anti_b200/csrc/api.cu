@@ -112,6 +112,7 @@ int64_t numel(const wqmm_tensor* t) {
 }
 
 bool contiguous(const wqmm_tensor* t) {
+  if (numel(t) == 0) return true;  // an empty tensor has no layout to check
   int64_t expect = 1;
   for (int i = t->ndim - 1; i >= 0; --i) {
     if (t->shape[i] != 1 && t->strides[i] != expect) return false;
@@ -391,8 +392,8 @@ extern "C" wqmm_status wqmm_get_workspace_size(const wqmm_tensor* x1, const wqmm
     int splits = 1;
     const int per_sm = ex->bn <= 64 ? 2 : 1;  // resident CTAs per SM (TMEM/shared-memory bound)
     const int64_t slots = static_cast<int64_t>(sms) * per_sm;
-    if (tiles < 4 * slots) {
-      // too few tiles to keep every SM streaming: split k (at least 8 k-steps per split)
+    if (tiles < slots) {
+      // too few tiles to occupy every SM: split k (at least 8 k-steps per split)
       const int64_t want = (4 * slots + tiles - 1) / tiles;
       const int64_t cap = kt / 8 > 1 ? kt / 8 : 1;
       splits = static_cast<int>(want < cap ? want : cap);
