@@ -6,6 +6,7 @@
 #include <chrono>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <new>
@@ -76,7 +77,10 @@ struct wqmm_executor {
   int group_size = 0;
   int num_groups = 0;
   int bn = 256;
-  int splits = 1;
+  int grid = 1;        // persistent CTAs of the GEMM
+  int stream_k = 0;    // 1: k steps of all tiles split evenly over the grid, partials + fix-up
+  int num_tiles = 0;
+  int max_slots = 0;
   // qmm
   const void* dq = nullptr;
   int dq_dtype = 0;
@@ -382,24 +386,40 @@ extern "C" wqmm_status wqmm_get_workspace_size(const wqmm_tensor* x1, const wqmm
   ex->num_groups = static_cast<int>(ng);
   uint64_t ws = 0;
   if (k > 0) {
-    // m tile: the smallest supported width that covers m (up to 256)
-    ex->bn = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <= 128 ? 128 : 256;
+    // m tile: the smallest supported width that covers m; large m uses 192
+    // (two TMEM accumulators fit, so the epilogue overlaps the next tile)
+    ex->bn = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <= 128 ? 128 : 192;
+    if (const char* env = std::getenv("WQMM_BN")) {  // tuning override
+      const int v = std::atoi(env);
+      if (v == 16 || v == 32 || v == 64 || v == 128 || v == 192 || v == 256) ex->bn = v;
+    }
     const int64_t num_mb = (m + ex->bn - 1) / ex->bn;
     const int64_t num_nb = (n + kWqNBlock - 1) / kWqNBlock;
-    const int kt = static_cast<int>((k + kWqKTile - 1) / kWqKTile);
+    const int64_t kt = (k + kWqKTile - 1) / kWqKTile;
     const int64_t tiles = num_mb * num_nb;
-    const int sms = sm_count();
-    int splits = 1;
-    const int per_sm = ex->bn <= 64 ? 2 : 1;  // resident CTAs per SM (TMEM/shared-memory bound)
-    const int64_t slots = static_cast<int64_t>(sms) * per_sm;
-    if (tiles < slots) {
-      // too few tiles to occupy every SM: split k (at least 8 k-steps per split)
-      const int64_t want = (4 * slots + tiles - 1) / tiles;
-      const int64_t cap = kt / 8 > 1 ? kt / 8 : 1;
-      splits = static_cast<int>(want < cap ? want : cap);
-      if (splits < 1) splits = 1;
+    if (tiles > 0x7FFFFFFFLL) {
+      delete ex;
+      return fail(WQMM_ERR_INNER_TILING, "too many output tiles");
     }
-    ex->splits = splits;
+    const int64_t slots = static_cast<int64_t>(sm_count()) * wqmm_ctas_per_sm(ex->bn, 0);
+    ex->num_tiles = static_cast<int>(tiles);
+    ex->stream_k = 0;
+    ex->grid = static_cast<int>(tiles < slots ? tiles : slots);
+    const char* sk_env = std::getenv("WQMM_STREAMK");
+    const bool force_sk = sk_env && std::atoi(sk_env) == 1;
+    const bool forbid_sk = sk_env && std::atoi(sk_env) == 0;
+    if (!forbid_sk && (force_sk || tiles < 2 * slots) && kt >= 2) {
+      // few tiles: spread all k steps evenly over one CTA per SM
+      ex->stream_k = 1;
+      const int64_t total = tiles * kt;
+      ex->grid = static_cast<int>(total < slots ? total : slots);
+      int ms = 1;
+      for (int64_t t = 0; t < tiles; ++t) {
+        const int64_t c = sk_owner(t * kt + kt - 1, total, ex->grid) - sk_owner(t * kt, total, ex->grid) + 1;
+        if (c > ms) ms = static_cast<int>(c);
+      }
+      ex->max_slots = ms;
+    }
     if (!ex->x2_packed) {
       ex->ws_pack = {ws, packed_bytes_for(x2->dtype, k, n, false)};
       ws = round_up(ws + ex->ws_pack.bytes, 256);
@@ -412,8 +432,8 @@ extern "C" wqmm_status wqmm_get_workspace_size(const wqmm_tensor* x1, const wqmm
         ws = round_up(ws + ex->ws_offset.bytes, 256);
       }
     }
-    if (splits > 1) {
-      ex->ws_partial = {ws, static_cast<uint64_t>(splits) * m * n * 4};
+    if (ex->stream_k) {
+      ex->ws_partial = {ws, static_cast<uint64_t>(tiles) * ex->max_slots * ex->bn * kWqNBlock * 4};
       ws = round_up(ws + ex->ws_partial.bytes, 256);
     }
   }
@@ -661,7 +681,7 @@ wqmm_status run_wqmm(void* ws, wqmm_executor* ex, cudaStream_t s) {
   p.bias = static_cast<const uint16_t*>(ex->bias);
   p.x3 = static_cast<const uint16_t*>(ex->x3);
   p.out = static_cast<uint16_t*>(ex->out);
-  p.partial = ex->splits > 1 ? reinterpret_cast<float*>(wsb + ex->ws_partial.offset) : nullptr;
+  p.partial = ex->stream_k ? reinterpret_cast<float*>(wsb + ex->ws_partial.offset) : nullptr;
   p.err = device_error_word();
   p.m = ex->m;
   p.n = ex->n;
@@ -669,28 +689,34 @@ wqmm_status run_wqmm(void* ws, wqmm_executor* ex, cudaStream_t s) {
   p.kt_total = (ex->k + kWqKTile - 1) / kWqKTile;
   p.num_nb = (ex->n + kWqNBlock - 1) / kWqNBlock;
   p.num_mb = static_cast<int>((ex->m + ex->bn - 1) / ex->bn);
-  p.splits = ex->splits;
+  p.num_tiles = ex->num_tiles;
+  p.stream_k = ex->stream_k;
+  p.max_slots = ex->max_slots;
   p.mode = ex->mode;
   p.group_size = ex->group_size;
   p.num_groups = ex->num_groups;
-  e = launch_wqmm_gemm(tmap, p, ex->bn, wk, bf16, s);
+  e = launch_wqmm_gemm(tmap, p, ex->bn, wk, bf16, ex->grid, s);
   if (e != cudaSuccess) return cuda_fail(e, "anti-quant GEMM launch");
-  if (ex->splits > 1) {
-    EpiParams ep{};
-    ep.partial = p.partial;
-    ep.scale = scale;
-    ep.offset = offset;
-    ep.bias = p.bias;
-    ep.x3 = p.x3;
-    ep.out = p.out;
-    ep.m = ex->m;
-    ep.n = ex->n;
-    ep.splits = ex->splits;
-    ep.mode = ex->mode;
-    ep.wk = wk;
-    ep.act_bf16 = bf16;
-    e = launch_wqmm_epilogue(ep, s);
-    if (e != cudaSuccess) return cuda_fail(e, "split-K epilogue launch");
+  if (ex->stream_k) {
+    FixupParams fp{};
+    fp.partial = p.partial;
+    fp.scale = scale;
+    fp.offset = offset;
+    fp.bias = p.bias;
+    fp.x3 = p.x3;
+    fp.out = p.out;
+    fp.m = ex->m;
+    fp.n = ex->n;
+    fp.bn = ex->bn;
+    fp.num_nb = p.num_nb;
+    fp.num_tiles = ex->num_tiles;
+    fp.kt_total = p.kt_total;
+    fp.grid = ex->grid;
+    fp.max_slots = ex->max_slots;
+    fp.mode = ex->mode;
+    fp.act_bf16 = bf16;
+    e = launch_wqmm_fixup(fp, s);
+    if (e != cudaSuccess) return cuda_fail(e, "stream-K fix-up launch");
   }
   return WQMM_SUCCESS;
 }

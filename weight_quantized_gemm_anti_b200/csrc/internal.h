@@ -32,17 +32,44 @@ struct WqParams {
   const uint16_t* bias;   // may be null
   const uint16_t* x3;     // may be null, (m, n)
   uint16_t* out;          // (m, n)
-  float* partial;         // split-K partials [splits][m][n], or null when splits == 1
+  float* partial;         // stream-K partial tiles [num_tiles][max_slots][BN][128] fp32, or null
   uint32_t* err;          // device error word
   int64_t m;
   int n, k;
   int kt_total;           // ceil(k / 64)
   int num_nb;             // ceil(n / 128)
   int num_mb;             // ceil(m / BN)
-  int splits;             // k splits
+  int num_tiles;          // num_mb * num_nb; tile t = (mb = t / num_nb, nb = t % num_nb)
+  int stream_k;           // 0: whole tiles round-robin over the grid; 1: k-steps split evenly
+  int max_slots;          // stream-K: partial slots per tile
   int mode;               // QuantMode
   int group_size;         // per-group only
   int num_groups;         // rows of scale/offset in per-group mode
+};
+
+// Stream-K ownership: with T = num_tiles * kt_total k-steps split over G CTAs,
+// CTA c owns steps [floor(c*T/G), floor((c+1)*T/G)); the owner of step s is
+// floor(((s+1)*G - 1) / T).  Shared by the GEMM and the fix-up kernel.
+__host__ __device__ inline int64_t sk_start(int64_t c, int64_t T, int64_t G) { return c * T / G; }
+__host__ __device__ inline int64_t sk_owner(int64_t s, int64_t T, int64_t G) { return ((s + 1) * G - 1) / T; }
+
+struct FixupParams {      // stream-K reduction + epilogue
+  const float* partial;
+  const uint16_t* scale;
+  const uint16_t* offset;
+  const uint16_t* bias;
+  const uint16_t* x3;
+  uint16_t* out;
+  int64_t m;
+  int n;
+  int bn;
+  int num_nb;
+  int num_tiles;
+  int kt_total;
+  int grid;
+  int max_slots;
+  int mode;
+  int act_bf16;
 };
 
 struct QParams {
@@ -91,8 +118,12 @@ struct EpiParams {        // split-K reduction + epilogue, and the k == 0 case
 // Launchers (return cudaSuccess or the launch error).
 cudaError_t launch_pack(const PackParams& p, cudaStream_t s);
 cudaError_t launch_transpose_u16(const uint16_t* src, uint16_t* dst, int rows, int cols, cudaStream_t s);
+// Launch configuration of the anti-quant GEMM for a BN-row m tile: CTAs per SM
+// the kernel's shared/tensor memory allows (the grid is a multiple of it).
+int wqmm_ctas_per_sm(int bn, int wk);
 cudaError_t launch_wqmm_gemm(const CUtensorMap& tmap_x1, const WqParams& p, int bn, int wk, bool act_bf16,
-                             cudaStream_t s);
+                             int grid, cudaStream_t s);
+cudaError_t launch_wqmm_fixup(const FixupParams& p, cudaStream_t s);
 cudaError_t launch_wqmm_epilogue(const EpiParams& p, cudaStream_t s);
 cudaError_t launch_qmm_gemm(const CUtensorMap& tmap_x1, const QParams& p, cudaStream_t s);
 

@@ -2,34 +2,45 @@
 //
 // Computes, per aclnnWeightQuantMatmulAllReduce "计算公式",
 //     out = x1 @ ((x2 + antiquantOffset) * antiquantScale) + bias + x3
-// as the transposed product  out^T = W^T x1^T  so that the dequantised weight
-// is the tcgen05 A operand held in tensor memory and x1 is the B operand in
-// shared memory:
+// as the transposed product  out^T = W^T x1^T,  so the dequantised weight is
+// the tcgen05 A operand held in tensor memory and x1 is the B operand in
+// shared memory.  A persistent, warp-specialised kernel, one CTA per SM:
 //
-//   * one CTA owns a tile of 128 weight columns (n) x BN activation rows (m);
-//     its accumulator D^T (128 lanes = n, BN columns = m, fp32) lives in TMEM;
-//   * warp 0 (one thread) streams, per 64-wide k step, the x1 tile (2-D tensor
-//     copy, 128-byte swizzle), the packed weight tile (one 1-D bulk copy) and,
-//     in per-group mode, the two scale/offset rows it needs, into a STAGES-deep
-//     shared-memory ring;
-//   * warps 2..5 (one per TMEM lane quadrant; thread = weight column n) unpack
-//     their column's 64 weights, dequantise them in registers and write them
-//     with tcgen05.st into one of four TMEM A stages;
-//   * warp 1 (one thread) issues four tcgen05.mma kind::f16 (M=128, N=BN, K=16)
-//     per k step, A from TMEM and B from shared memory, and releases the
-//     shared-memory and TMEM stages with tcgen05.commit;
-//   * after the last k step warps 2..5 read the accumulator back with
-//     tcgen05.ld and apply the epilogue (scale, + bias, + x3, round) -- or
-//     store fp32 split-K partials that a second kernel reduces in fixed order.
+//   warp 0      x1 producer: per 64-wide k step, the x1 tile (one 2-D tensor
+//               copy, 128-byte swizzle) into the x1 ring, which the MMA reads;
+//   warp 6      weight producer: the packed 128-column weight tile (one 1-D
+//               bulk copy) into the weight ring, which the dequantisers read
+//               and release as soon as the tile is in registers -- so weights
+//               stream far ahead of the MMA while x1 tiles wait for it;
+//   warp 1      MMA issuer: four tcgen05.mma kind::f16 (M=128, N=BN, K=16) per
+//               k step, A from TMEM, B from shared memory, fp32 accumulators in
+//               TMEM (two buffers when they fit, so the epilogue of one tile
+//               overlaps the main loop of the next); stages are released with
+//               tcgen05.commit;
+//   warps 2..5  epilogue (one per TMEM lane quadrant): tcgen05.ld of the
+//               accumulator, fp32 scale / + bias / + x3, one rounding, store --
+//               or an fp32 partial tile in stream-K mode;
+//   warps 7..   DG dequantisation groups of four warps (one per lane
+//               quadrant; thread = weight column).  Group g takes the k steps
+//               g, g+DG, ...: loads its column's per-group scale/offset from
+//               L2 one step ahead, unpacks its column's 64 weights, dequantises them
+//               in registers and tcgen05.st's them into one of its own TMEM A
+//               stages, so DG k steps are dequantised concurrently.
 //
-// Dequantisation (per element pair, bf16x2 / f16x2 registers):
-//   int4, integer offset:   t = 0x4300|nibble (=128+q+8, exact); v = t + (off-136)
-//                            (exact); per-group w = v * s (one rounding);
-//                            per-tensor/channel w = v, scale applied in fp32 later.
-//   int8: built exactly in fp32 (0x4B000000|byte trick), same split.
-//   fp8-e4m3: converted exactly; scale applied in fp32 in the epilogue.
-//   Non-integer offsets take an fp32 path: w = round((q + off) * s).
-// No cluster multicast; every wait is bounded (ptx.cuh).
+// Work is either whole output tiles dealt round-robin to the CTAs, or (few
+// tiles: small m) all k steps of all tiles split evenly over the CTAs
+// ("stream-K"); then every CTA writes fp32 partial tiles and a second kernel
+// sums them in a fixed order (deterministic, no inter-CTA waiting).
+//
+// Dequantisation, per element pair in bf16x2 / f16x2 registers:
+//   int4, integer offsets (warp-uniform test): t = 0x4300|nibble (= 128+q+8)
+//       then v = t + (off - 136), exact; per-group w = v * s (one rounding);
+//       per-tensor/per-channel w = v and the scale is applied to the fp32
+//       accumulator in the epilogue.
+//   int8: built exactly in fp32 from 0x4B000000|byte, same split of the scale.
+//   fp8-e4m3: converted exactly, scale in the epilogue.
+//   other offsets: fp32 path, w = round((q + off) * s), epilogue scale 1.
+// No cluster multicast anywhere; every wait is bounded (ptx.cuh).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -41,22 +52,34 @@ namespace wqmm {
 
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kAStages = 4;
-constexpr int kSoBytes = 1024;  // per stage: 2 half-steps x (scale, offset) x 128 x 2 B
+constexpr unsigned kFull = 0xFFFFFFFFu;
 
-template <int BN>
+constexpr int pow2ceil(int v) { return v <= 32 ? 32 : v <= 64 ? 64 : v <= 128 ? 128 : v <= 256 ? 256 : 512; }
+constexpr int cmin(int a, int b) { return a < b ? a : b; }
+
+constexpr int cmax(int a, int b) { return a > b ? a : b; }
+
+template <int BN, int DG, int WK>
 struct Cfg {
-  static constexpr int kStages = BN >= 256 ? 5 : (BN >= 128 ? 7 : 10);
+  static constexpr int kTile = wq_tile_bytes(WK);
   static constexpr int kX1Bytes = BN * 128;
   static constexpr int kAccCols = BN < 32 ? 32 : BN;
-  static constexpr int kTmemNeed = kAccCols + kAStages * 32;
-  static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
-                                   : kTmemNeed <= 256 ? 256 : 512;
-  template <int WK>
-  static constexpr int smem_bytes() {
-    return kStages * (kX1Bytes + wq_tile_bytes(WK) + kSoBytes) + 1024;
-  }
+  static constexpr int kNAcc = (2 * kAccCols + 4 * 32 <= 512) ? 2 : 1;
+  static constexpr int kACol0 = kNAcc * kAccCols;
+  // TMEM A stages: as many as fit (up to 8), a multiple of DG so that every
+  // dequantisation group owns its own stages
+  static constexpr int kAStages = cmin(8, (512 - kACol0) / 32 / DG * DG);
+  static constexpr int kTmemCols = pow2ceil(kACol0 + kAStages * 32);
+  // shared memory: an x1 ring (read by the MMA) and a weight ring (read by the
+  // dequantisers, released as soon as a tile is in registers)
+  static constexpr int kSmemBudget = 200 * 1024;
+  static constexpr int kXStages = cmin(16, cmax(4, (kSmemBudget * 3 / 5) / kX1Bytes));
+  static constexpr int kWStages = cmin(32, (kSmemBudget - kXStages * kX1Bytes) / kTile);
+  static constexpr int kThreads = 32 * (7 + 4 * DG);
+  static constexpr int kSmemBytes = kXStages * kX1Bytes + kWStages * kTile + 1024;
+  static_assert(kAStages >= DG && kAStages % DG == 0, "A stages");
+  static_assert(kACol0 + kAStages * 32 <= 512, "TMEM budget");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
 __device__ __forceinline__ float act_f32(uint16_t v, bool bf16) {
@@ -67,10 +90,10 @@ __device__ __forceinline__ uint16_t f32_act(float v, bool bf16) {
   return bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(v)) : __half_as_ushort(__float2half_rn(v));
 }
 
+// Offsets that are small integers fold exactly into the operand: q + off is an
+// integer of magnitude < 256, exact in bf16 and f16.
 __device__ __forceinline__ bool small_int(float off) { return off == rintf(off) && fabsf(off) <= 112.f; }
 
-// Pack two fp32 into a bf16x2 / f16x2 register, round to nearest even; `lo`
-// lands in bits 0..15.
 template <bool BF16>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   uint32_t r;
@@ -101,136 +124,260 @@ __device__ __forceinline__ uint32_t mul2(uint32_t a, uint32_t b) {
   return r;
 }
 
-template <bool BF16>
-__device__ __forceinline__ uint32_t splat(float v) {
-  return pack2<BF16>(v, v);
+__device__ __forceinline__ uint32_t splat_bits(uint16_t b) {
+  return static_cast<uint32_t>(b) | (static_cast<uint32_t>(b) << 16);
 }
 
-// Per-half-step dequantisation constants for one weight column.
-struct DqConst {
-  uint32_t c2;     // (offset - magic) splatted, exact (integer path)
-  uint32_t s2;     // scale splatted (per-group integer path)
-  float off, s;    // fp32 values (general path)
-  bool fast;       // integer offset: exact add path
-  bool apply_s;    // multiply by the scale in the operand (per-group or non-integer offset)
-};
-
-template <bool BF16, int WK>
-__device__ __forceinline__ DqConst make_const(float s, float off, bool per_group) {
-  DqConst c;
-  c.off = off;
-  c.s = s;
-  c.fast = small_int(off);
-  c.apply_s = per_group || !c.fast;
-  // int4 magic: bf16 0x4300 = 128, f16 0x6400 = 1024; stored nibble = q + 8.
-  const float magic = (WK == kW4) ? (BF16 ? 136.f : 1032.f) : (BF16 ? 0.f : 1152.f);
-  c.c2 = splat<BF16>(off - magic);
-  c.s2 = splat<BF16>(s);
-  return c;
-}
-
-// Dequantise the 32 k values of one 16-byte int4 chunk into 16 operand registers.
-template <bool BF16>
-__device__ __forceinline__ void dq_int4(const uint4 chunk, const DqConst& c, uint32_t* out) {
-  const uint32_t words[4] = {chunk.x, chunk.y, chunk.z, chunk.w};
-  const uint32_t magic = BF16 ? 0x43004300u : 0x64006400u;
+// ---------------------------------------------------------------- int4
+// 16-byte chunk = 32 k values -> 16 operand registers (k pairs).
+// Exact integer path: v = (0x4300|nibble pair) + c2, optionally * s2.
+template <bool BF16, bool MUL>
+__device__ __forceinline__ void dq4_fast(const uint4 ch, uint32_t c2, uint32_t s2, uint32_t* out) {
+  const uint32_t words[4] = {ch.x, ch.y, ch.z, ch.w};
+  constexpr uint32_t kMagic = BF16 ? 0x43004300u : 0x64006400u;
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const uint32_t t = ((words[w] >> (4 * j)) & 0x000F000Fu) | magic;
-      uint32_t v;
-      if (c.fast) {
-        v = add2<BF16>(t, c.c2);
-        if (c.apply_s) v = mul2<BF16>(v, c.s2);
-      } else {
-        float lo, hi;
-        if constexpr (BF16) {
-          lo = __uint_as_float(t << 16) - 136.f;
-          hi = __uint_as_float(t & 0xFFFF0000u) - 136.f;
-        } else {
-          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&t));
-          lo = f.x - 1032.f;
-          hi = f.y - 1032.f;
-        }
-        v = pack2<BF16>((lo + c.off) * c.s, (hi + c.off) * c.s);
-      }
+      const uint32_t t = ((words[w] >> (4 * j)) & 0x000F000Fu) | kMagic;
+      uint32_t v = add2<BF16>(t, c2);
+      if constexpr (MUL) v = mul2<BF16>(v, s2);
       out[4 * w + j] = v;
     }
   }
 }
 
-// Dequantise the 16 k values of one 16-byte int8 chunk into 8 operand registers.
+// General path: w = round((q + off) * s) through fp32.
 template <bool BF16>
-__device__ __forceinline__ void dq_int8(const uint4 chunk, const DqConst& c, uint32_t* out) {
-  const uint32_t words[4] = {chunk.x, chunk.y, chunk.z, chunk.w};
+__device__ __forceinline__ void dq4_general(const uint4 ch, float off, float s, uint32_t* out) {
+  const uint32_t words[4] = {ch.x, ch.y, ch.z, ch.w};
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t u = (words[w] >> (4 * j)) & 0x000F000Fu;  // two biased nibbles (q + 8)
+      const float lo = static_cast<float>(static_cast<int>(u & 0xFu) - 8);
+      const float hi = static_cast<float>(static_cast<int>(u >> 16) - 8);
+      out[4 * w + j] = pack2<BF16>((lo + off) * s, (hi + off) * s);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- int8
+// 16-byte chunk = 16 k values (biased bytes q + 128) -> 8 operand registers.
+template <bool BF16, bool MUL>
+__device__ __forceinline__ void dq8_fast(const uint4 ch, float off, float s, uint32_t c2, uint32_t s2,
+                                         uint32_t* out) {
+  const uint32_t words[4] = {ch.x, ch.y, ch.z, ch.w};
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       uint32_t v;
-      if (!BF16 && c.fast) {
-        // f16: 0x6400 | byte = 1024 + (q + 128); add (off - 1152) exactly.
+      if constexpr (!BF16) {
+        // f16: 0x6400 | byte = 1024 + q + 128 exactly; add (off - 1152) exactly.
         const uint32_t t = __byte_perm(words[w], 0x64646464u, h ? 0x7372 : 0x7170);
-        v = add2<false>(t, c.c2);
-        if (c.apply_s) v = mul2<false>(v, c.s2);
+        v = add2<false>(t, c2);
+        if constexpr (MUL) v = mul2<false>(v, s2);
       } else {
-        // fp32: 0x4B000000 | byte = 2^23 + q + 128, exact.
-        const float lo = __uint_as_float(0x4B000000u | ((words[w] >> (16 * h)) & 0xFFu)) - 8388736.f;
-        const float hi = __uint_as_float(0x4B000000u | ((words[w] >> (16 * h + 8)) & 0xFFu)) - 8388736.f;
-        if (c.apply_s)
-          v = pack2<BF16>((lo + c.off) * c.s, (hi + c.off) * c.s);
-        else
-          v = pack2<BF16>(lo + c.off, hi + c.off);
+        // fp32: 0x4B000000 | byte = 2^23 + q + 128; subtracting (2^23 + 128 - off) is exact.
+        const float base = 8388736.f - off;
+        const float lo = __uint_as_float(__byte_perm(words[w], 0x4B000000u, h ? 0x7442 : 0x7440)) - base;
+        const float hi = __uint_as_float(__byte_perm(words[w], 0x4B000000u, h ? 0x7443 : 0x7441)) - base;
+        v = MUL ? pack2<true>(lo * s, hi * s) : pack2<true>(lo, hi);
       }
       out[2 * w + h] = v;
     }
   }
 }
 
-// Convert the 16 fp8-e4m3 values of one chunk exactly (no offset, scale later).
 template <bool BF16>
-__device__ __forceinline__ void dq_fp8(const uint4 chunk, uint32_t* out) {
-  const uint32_t words[4] = {chunk.x, chunk.y, chunk.z, chunk.w};
+__device__ __forceinline__ void dq8_general(const uint4 ch, float off, float s, uint32_t* out) {
+  const uint32_t words[4] = {ch.x, ch.y, ch.z, ch.w};
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float lo = static_cast<float>(static_cast<int>((words[w] >> (16 * h)) & 0xFFu) - 128);
+      const float hi = static_cast<float>(static_cast<int>((words[w] >> (16 * h + 8)) & 0xFFu) - 128);
+      out[2 * w + h] = pack2<BF16>((lo + off) * s, (hi + off) * s);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- fp8-e4m3
+template <bool BF16>
+__device__ __forceinline__ void dq_fp8(const uint4 ch, uint32_t* out) {
+  const uint32_t words[4] = {ch.x, ch.y, ch.z, ch.w};
 #pragma unroll
   for (int w = 0; w < 4; ++w) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>((words[w] >> (16 * h)) & 0xFFFFu);
       const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
-      uint32_t v;
       if constexpr (BF16) {
         const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
-        v = pack2<true>(f.x, f.y);
+        out[2 * w + h] = pack2<true>(f.x, f.y);
       } else {
-        v = static_cast<uint32_t>(hr.x) | (static_cast<uint32_t>(hr.y) << 16);
+        out[2 * w + h] = static_cast<uint32_t>(hr.x) | (static_cast<uint32_t>(hr.y) << 16);
       }
-      out[2 * w + h] = v;
     }
   }
 }
 
-template <int BN, int WK, bool BF16>
-__global__ void __launch_bounds__(kThreads, 1)
+// ---------------------------------------------------------------- per-group halves
+// Half H (32 k values) of a k step in per-group mode, given the raw scale and
+// offset bits of this column's group row for that half (0 for a half past k
+// or a column past n: those weights become 0).
+template <bool BF16, int H>
+__device__ __forceinline__ void dq4_group_half(const uint4 ch, uint16_t sb, uint16_t ob, uint32_t* a) {
+  const float off = act_f32(ob, BF16);
+  if (__all_sync(kFull, small_int(off))) {
+    const float c = off - (BF16 ? 136.f : 1032.f);
+    dq4_fast<BF16, true>(ch, pack2<BF16>(c, c), splat_bits(sb), a + 16 * H);
+  } else {
+    dq4_general<BF16>(ch, off, act_f32(sb, BF16), a + 16 * H);
+  }
+}
+
+template <bool BF16, int H>
+__device__ __forceinline__ void dq8_group_half(const uint4 chA, const uint4 chB, uint16_t sb, uint16_t ob,
+                                               uint32_t* a) {
+  const float s = act_f32(sb, BF16);
+  const float off = act_f32(ob, BF16);
+  if (__all_sync(kFull, small_int(off))) {
+    const float c = off - 1152.f;
+    const uint32_t c2 = pack2<BF16>(c, c);
+    dq8_fast<BF16, true>(chA, off, s, c2, splat_bits(sb), a + 16 * H);
+    dq8_fast<BF16, true>(chB, off, s, c2, splat_bits(sb), a + 16 * H + 8);
+  } else {
+    dq8_general<BF16>(chA, off, s, a + 16 * H);
+    dq8_general<BF16>(chB, off, s, a + 16 * H + 8);
+  }
+}
+
+// Scale/offset bits of one column for the two 32-wide halves of a k step
+// (per-group mode).
+struct GroupSO {
+  uint16_t s[2], o[2];
+};
+
+// Group row of half index hidx = 2*kt (+1 for the second half): row = hidx / gq,
+// gq = G / 32 halves per group.  Advanced without division along a group's
+// k steps.
+struct GroupRow {
+  int row, rem;
+  __device__ __forceinline__ void init(int hidx, int gq) {
+    row = hidx / gq;
+    rem = hidx - row * gq;
+  }
+  __device__ __forceinline__ void advance(int halves, int gq) {
+    rem += halves;
+    while (rem >= gq) {
+      rem -= gq;
+      ++row;
+    }
+  }
+  __device__ __forceinline__ int row1(int gq) const { return row + (rem + 1 >= gq ? 1 : 0); }
+};
+
+__device__ __forceinline__ GroupSO load_group_so(const WqParams& p, int kt, const GroupRow& gr, int gq, int nn,
+                                                 bool col_ok) {
+  GroupSO r;
+  const int rows[2] = {gr.row, gr.row1(gq)};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const bool use = col_ok && (kt * kWqKTile + 32 * h < p.k);
+    const int64_t idx = static_cast<int64_t>(rows[h]) * p.n + nn;
+    r.s[h] = use ? __ldg(p.scale + idx) : uint16_t(0);
+    r.o[h] = (use && p.offset) ? __ldg(p.offset + idx) : uint16_t(0);
+  }
+  return r;
+}
+
+// ---------------------------------------------------------------- schedule
+struct Item {
+  int tile, kt0, kt1, slot;  // slot < 0: whole tile, write the output
+};
+
+// Identical walk of this CTA's work in every role.
+struct Walker {
+  int64_t cur, end, T;
+  __device__ __forceinline__ void init(const WqParams& p) {
+    if (p.stream_k) {
+      T = static_cast<int64_t>(p.num_tiles) * p.kt_total;
+      cur = sk_start(blockIdx.x, T, gridDim.x);
+      end = sk_start(blockIdx.x + 1, T, gridDim.x);
+    } else {
+      T = 0;
+      cur = blockIdx.x;
+      end = p.num_tiles;
+    }
+  }
+  __device__ __forceinline__ bool next(const WqParams& p, Item& it) {
+    if (cur >= end) return false;
+    if (!p.stream_k) {
+      it.tile = static_cast<int>(cur);
+      it.kt0 = 0;
+      it.kt1 = p.kt_total;
+      it.slot = -1;
+      cur += gridDim.x;
+      return true;
+    }
+    const int64_t tile = cur / p.kt_total;
+    const int64_t tile_end = (tile + 1) * p.kt_total;
+    const int64_t e = end < tile_end ? end : tile_end;
+    it.tile = static_cast<int>(tile);
+    it.kt0 = static_cast<int>(cur - tile * p.kt_total);
+    it.kt1 = it.kt0 + static_cast<int>(e - cur);
+    it.slot = static_cast<int>(blockIdx.x - sk_owner(tile * p.kt_total, T, gridDim.x));
+    cur = e;
+    return true;
+  }
+};
+
+// Per-column constants of per-tensor / per-channel modes for one tile.
+struct ColConst {
+  float s, off;
+  uint32_t c2;
+  bool fast;  // warp-uniform: every column of this warp has a small-integer offset
+};
+
+template <bool BF16, int WK>
+__device__ __forceinline__ ColConst col_const(const WqParams& p, int nn, bool col_ok) {
+  ColConst c;
+  const int idx = (p.mode == kPerTensor) ? 0 : (col_ok ? nn : 0);
+  c.s = act_f32(p.scale[idx], BF16);
+  c.off = p.offset ? act_f32(p.offset[idx], BF16) : 0.f;
+  c.fast = __all_sync(kFull, small_int(c.off));
+  const float magic = (WK == kW4) ? (BF16 ? 136.f : 1032.f) : (BF16 ? 0.f : 1152.f);
+  c.c2 = pack2<BF16>(c.off - magic, c.off - magic);
+  return c;
+}
+
+template <int BN, int DG, int WK, bool BF16>
+__global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
     wqmm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x1, const WqParams p) {
-  using C = Cfg<BN>;
-  constexpr int S = C::kStages;
-  constexpr int kTile = wq_tile_bytes(WK);
+  using C = Cfg<BN, DG, WK>;
+  constexpr int SX = C::kXStages;
+  constexpr int SW = C::kWStages;
+  constexpr int AS = C::kAStages;
+  constexpr int kTile = C::kTile;
   constexpr uint32_t kIdesc = idesc_make(1u, BF16 ? 1u : 0u, 128u, static_cast<uint32_t>(BN));
-  constexpr uint32_t kAccCol = 0;
-  constexpr uint32_t kACol0 = C::kAccCols;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* s_x1 = smem;
-  uint8_t* s_w = s_x1 + S * C::kX1Bytes;
-  uint8_t* s_so = s_w + S * kTile;
+  uint8_t* s_x1 = smem;                  // SX x (BN x 128 B), 1024-aligned slabs
+  uint8_t* s_w = s_x1 + SX * C::kX1Bytes;  // SW x packed weight tile
 
-  __shared__ __align__(8) uint64_t bar_full[S];
-  __shared__ __align__(8) uint64_t bar_empty[S];
-  __shared__ __align__(8) uint64_t bar_afull[kAStages];
-  __shared__ __align__(8) uint64_t bar_aempty[kAStages];
-  __shared__ __align__(8) uint64_t bar_acc;
+  __shared__ __align__(8) uint64_t bar_xfull[SX];
+  __shared__ __align__(8) uint64_t bar_xempty[SX];
+  __shared__ __align__(8) uint64_t bar_wfull[SW];
+  __shared__ __align__(8) uint64_t bar_wempty[SW];
+  __shared__ __align__(8) uint64_t bar_afull[AS];
+  __shared__ __align__(8) uint64_t bar_aempty[AS];
+  __shared__ __align__(8) uint64_t bar_accfull[2];
+  __shared__ __align__(8) uint64_t bar_accempty[2];
   __shared__ __align__(8) uint64_t bar_drain;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
@@ -238,28 +385,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // tile coordinates: split fastest, then n-block, then m-block
-  int bid = blockIdx.x;
-  const int split = bid % p.splits;
-  bid /= p.splits;
-  const int nb = bid % p.num_nb;
-  const int mb = bid / p.num_nb;
-  const int kt_begin = static_cast<int>((static_cast<int64_t>(split) * p.kt_total) / p.splits);
-  const int kt_end = static_cast<int>((static_cast<int64_t>(split + 1) * p.kt_total) / p.splits);
-  const int n_iter = kt_end - kt_begin;
-  const int n0 = nb * kWqNBlock;
-  const int64_t m0 = static_cast<int64_t>(mb) * BN;
-
   if (threadIdx.x == 0) {
-    for (int i = 0; i < S; ++i) {
-      mbar_init(&bar_full[i], 1);
-      mbar_init(&bar_empty[i], 4 + 1);
+    for (int i = 0; i < SX; ++i) {
+      mbar_init(&bar_xfull[i], 1);
+      mbar_init(&bar_xempty[i], 1);
     }
-    for (int i = 0; i < kAStages; ++i) {
+    for (int i = 0; i < SW; ++i) {
+      mbar_init(&bar_wfull[i], 1);
+      mbar_init(&bar_wempty[i], 4);
+    }
+    for (int i = 0; i < AS; ++i) {
       mbar_init(&bar_afull[i], 4);
       mbar_init(&bar_aempty[i], 1);
     }
-    mbar_init(&bar_acc, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_accfull[i], 1);
+      mbar_init(&bar_accempty[i], 4);
+    }
     mbar_init(&bar_drain, 1);
     abort_sh = 0;
     fence_barrier_init();
@@ -274,186 +416,221 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = tmem_base_sh;
   volatile int* abort_flag = &abort_sh;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  Walker walk;
+  walk.init(p);
+  Item it;
+
+  if (warp == 0 || warp == 6) {
+    // ============================================================ producers
+    // warp 0: x1 tiles (one 2-D tensor copy per k step) for the MMA;
+    // warp 6: packed weight tiles (one 1-D bulk copy per k step) for the dequantisers.
     if (lane == 0) {
-      prefetch_tensormap(&tmap_x1);
-      const bool grp = (p.mode == kPerGroup);
-      int issued = 0;
-      for (int i = 0; i < n_iter; ++i) {
-        const int st = i % S;
-        const uint32_t ph = (i / S) & 1;
-        if (!mbar_wait(&bar_empty[st], ph ^ 1, abort_flag, p.err, kDevTimeoutProducer)) break;
-        const int kt = kt_begin + i;
-        // scale/offset rows of the two 32-wide half-steps (per-group only)
-        int grow[2] = {-1, -1};
-        uint32_t so_bytes = 0;
-        const int ncols = min(kWqNBlock, p.n - n0);
-        if (grp) {
-          for (int h = 0; h < 2; ++h) {
-            const int kk = kt * kWqKTile + 32 * h;
-            if (kk < p.k) grow[h] = kk / p.group_size;
+      const bool is_x = (warp == 0);
+      if (is_x) prefetch_tensormap(&tmap_x1);
+      const int ns = is_x ? SX : SW;
+      uint64_t* full = is_x ? bar_xfull : bar_wfull;
+      uint64_t* empty = is_x ? bar_xempty : bar_wempty;
+      uint32_t g = 0;
+      bool live = true;
+      while (live && walk.next(p, it)) {
+        const int nb = it.tile % p.num_nb;
+        const int32_t m0 = static_cast<int32_t>(static_cast<int64_t>(it.tile / p.num_nb) * BN);
+        for (int kt = it.kt0; kt < it.kt1; ++kt, ++g) {
+          const int st = g % ns;
+          if (!mbar_wait(&empty[st], ((g / ns) & 1) ^ 1, abort_flag, p.err, kDevTimeoutProducer)) {
+            live = false;
+            break;
           }
-          for (int h = 0; h < 2; ++h)
-            if (grow[h] >= 0) so_bytes += static_cast<uint32_t>(ncols) * 2u * (p.offset ? 2u : 1u);
-        }
-        mbar_arrive_expect_tx(&bar_full[st], static_cast<uint32_t>(C::kX1Bytes + kTile) + so_bytes);
-        tma_load_2d(s_x1 + st * C::kX1Bytes, &tmap_x1, &bar_full[st], kt * kWqKTile, static_cast<int32_t>(m0));
-        bulk_g2s(s_w + st * kTile,
-                 p.wpack + (static_cast<int64_t>(nb) * p.kt_total + kt) * kTile, kTile, &bar_full[st]);
-        if (grp) {
-          uint8_t* so = s_so + st * kSoBytes;
-          for (int h = 0; h < 2; ++h) {
-            if (grow[h] < 0) continue;
-            const uint16_t* srow = p.scale + static_cast<int64_t>(grow[h]) * p.n + n0;
-            bulk_g2s(so + h * 512, srow, ncols * 2, &bar_full[st]);
-            if (p.offset) {
-              const uint16_t* orow = p.offset + static_cast<int64_t>(grow[h]) * p.n + n0;
-              bulk_g2s(so + h * 512 + 256, orow, ncols * 2, &bar_full[st]);
-            }
+          if (is_x) {
+            mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(C::kX1Bytes));
+            tma_load_2d(s_x1 + st * C::kX1Bytes, &tmap_x1, &full[st], kt * kWqKTile, m0);
+          } else {
+            mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(kTile));
+            bulk_g2s(s_w + st * kTile, p.wpack + (static_cast<int64_t>(nb) * p.kt_total + kt) * kTile, kTile,
+                     &full[st]);
           }
         }
-        ++issued;
       }
-      // drain: wait until every copy issued into the ring has landed
-      for (int i = (issued > S ? issued - S : 0); i < issued; ++i) {
+      // every copy issued into the ring has landed before the CTA may exit
+      const uint32_t first = g > static_cast<uint32_t>(ns) ? g - ns : 0;
+      for (uint32_t i = first; i < g; ++i) {
         volatile int no_abort = 0;
-        mbar_wait(&bar_full[i % S], (i / S) & 1, &no_abort, p.err, kDevTimeoutDrain);
+        mbar_wait(&full[i % ns], (i / ns) & 1, &no_abort, p.err, kDevTimeoutDrain);
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ============================================================ MMA issuer
     if (lane == 0) {
-      for (int i = 0; i < n_iter; ++i) {
-        const int st = i % S;
-        const int as = i % kAStages;
-        if (!mbar_wait(&bar_full[st], (i / S) & 1, abort_flag, p.err, kDevTimeoutMma)) break;
-        if (!mbar_wait(&bar_afull[as], (i / kAStages) & 1, abort_flag, p.err, kDevTimeoutMma)) break;
+      uint32_t g = 0, j = 0;
+      bool live = true;
+      while (live && walk.next(p, it)) {
+        const int ab = j % C::kNAcc;
+        if (!mbar_wait(&bar_accempty[ab], ((j / C::kNAcc) & 1) ^ 1, abort_flag, p.err, kDevTimeoutMma)) break;
         tc_fence_after();
-        const uint32_t b_base = smem_u32(s_x1 + st * C::kX1Bytes);
+        const uint32_t d_tmem = tmem + ab * C::kAccCols;
+        for (int kt = it.kt0; kt < it.kt1; ++kt, ++g) {
+          const int sx = g % SX;
+          const int as = g % AS;
+          if (!mbar_wait(&bar_xfull[sx], (g / SX) & 1, abort_flag, p.err, kDevTimeoutMma) ||
+              !mbar_wait(&bar_afull[as], (g / AS) & 1, abort_flag, p.err, kDevTimeoutMma)) {
+            live = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t b_base = smem_u32(s_x1 + sx * C::kX1Bytes);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bdesc = sdesc_kmajor_sw128(b_base + kk * 32);
-          const uint32_t a_tmem = tmem + kACol0 + as * 32 + kk * 8;
-          mma_f16_ts(tmem + kAccCol, a_tmem, bdesc, kIdesc, (i > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {
+            mma_f16_ts(d_tmem, tmem + C::kACol0 + as * 32 + kk * 8, sdesc_kmajor_sw128(b_base + kk * 32), kIdesc,
+                       (kt > it.kt0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&bar_xempty[sx]);
+          mma_commit(&bar_aempty[as]);
         }
-        mma_commit(&bar_empty[st]);
-        mma_commit(&bar_aempty[as]);
+        if (!live) break;
+        mma_commit(&bar_accfull[ab]);
+        ++j;
       }
-      mma_commit(&bar_acc);
-      // wait for every MMA this thread issued before the TMEM is released
       mma_commit(&bar_drain);
       volatile int no_abort = 0;
       mbar_wait(&bar_drain, 0, &no_abort, p.err, kDevTimeoutDrain);
     }
-  } else {
-    // ------------------------------------------------------------ dequant + epilogue
-    const int quad = warp & 3;                       // TMEM lane quadrant this warp may access
-    const int r = quad * 32 + lane;                  // row of the 128-column weight block
-    const int nn = n0 + r;
-    const bool col_ok = nn < p.n;
+  } else if (warp < 6) {
+    // ============================================================ epilogue
+    const int quad = warp & 3;
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
-    // per-tensor / per-channel constants, fixed for the whole tile
-    DqConst cst{};
-    if (p.mode != kPerGroup) {
-      const int idx = (p.mode == kPerTensor) ? 0 : (col_ok ? nn : 0);
-      const float s = act_f32(p.scale[idx], BF16);
-      const float off = p.offset ? act_f32(p.offset[idx], BF16) : 0.f;
-      cst = make_const<BF16, WK>(s, off, false);
-    }
-    bool ok = true;
-    for (int i = 0; i < n_iter && ok; ++i) {
-      const int st = i % S;
-      const int as = i % kAStages;
-      bool got = mbar_wait(&bar_full[st], (i / S) & 1, abort_flag, p.err, kDevTimeoutDequant);
-      got = got && mbar_wait(&bar_aempty[as], ((i / kAStages) & 1) ^ 1, abort_flag, p.err, kDevTimeoutDequant);
-      // tcgen05.st below is warp-collective: proceed only if every lane's wait succeeded
-      if (!__all_sync(0xFFFFFFFFu, got)) {
-        ok = false;
-        break;
-      }
-      const uint8_t* wt = s_w + st * kTile;
-      const int kbase = (kt_begin + i) * kWqKTile;
-      uint32_t a[32];
-      if constexpr (WK == kW4) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          DqConst c = cst;
-          if (p.mode == kPerGroup) {
-            // a half-step past k has no scale/offset row staged: its weights become 0
-            const bool use = col_ok && (kbase + 32 * h < p.k);
-            const uint8_t* so = s_so + st * kSoBytes + h * 512;
-            const float s = use ? act_f32(reinterpret_cast<const uint16_t*>(so)[r], BF16) : 0.f;
-            const float off =
-                (p.offset && use) ? act_f32(reinterpret_cast<const uint16_t*>(so + 256)[r], BF16) : 0.f;
-            c = make_const<BF16, WK>(s, off, true);
-          }
-          const uint4 chunk = *reinterpret_cast<const uint4*>(wt + (h * kWqNBlock + r) * 16);
-          dq_int4<BF16>(chunk, c, a + 16 * h);
-        }
-      } else {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 chunk = *reinterpret_cast<const uint4*>(wt + (q * kWqNBlock + r) * 16);
-          if constexpr (WK == kWFp8) {
-            dq_fp8<BF16>(chunk, a + 8 * q);
-          } else {
-            DqConst c = cst;
-            if (p.mode == kPerGroup) {
-              const bool use = col_ok && (kbase + 32 * (q >> 1) < p.k);
-              const uint8_t* so = s_so + st * kSoBytes + (q >> 1) * 512;
-              const float s = use ? act_f32(reinterpret_cast<const uint16_t*>(so)[r], BF16) : 0.f;
-              const float off =
-                  (p.offset && use) ? act_f32(reinterpret_cast<const uint16_t*>(so + 256)[r], BF16) : 0.f;
-              c = make_const<BF16, WK>(s, off, true);
-            }
-            dq_int8<BF16>(chunk, c, a + 8 * q);
-          }
-        }
-      }
-      tmem_st_x32(tmem + lane_addr + kACol0 + as * 32, a);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&bar_afull[as]);
-        mbar_arrive(&bar_empty[st]);
-      }
-    }
-    // epilogue: wait for the accumulator (warp-uniform outcome before tcgen05.ld)
-    bool acc_ready = ok && n_iter > 0 && mbar_wait(&bar_acc, 0, abort_flag, p.err, kDevTimeoutEpilogue);
-    acc_ready = __all_sync(0xFFFFFFFFu, acc_ready && !*abort_flag);
-    if (acc_ready) {
+    uint32_t j = 0;
+    while (walk.next(p, it)) {
+      const int ab = j % C::kNAcc;
+      bool ready = mbar_wait(&bar_accfull[ab], (j / C::kNAcc) & 1, abort_flag, p.err, kDevTimeoutEpilogue);
+      if (!__all_sync(kFull, ready && !*abort_flag)) break;
       tc_fence_after();
-      float escale = 1.f;
-      if (p.mode != kPerGroup && WK != kWFp8) escale = cst.apply_s ? 1.f : cst.s;
-      if (WK == kWFp8) escale = cst.s;
-      const float bias_v = (p.bias && col_ok && p.splits == 1) ? act_f32(p.bias[nn], BF16) : 0.f;
-      constexpr int kChunk = BN < 32 ? BN : 32;
+      const int nb = it.tile % p.num_nb;
+      const int64_t m0 = static_cast<int64_t>(it.tile / p.num_nb) * BN;
+      const int nl = quad * 32 + lane;  // column within the tile
+      const int nn = nb * kWqNBlock + nl;
+      const bool col_ok = nn < p.n;
+      float escale = 1.f, bias_v = 0.f;
+      if (it.slot < 0) {
+        if (p.mode != kPerGroup) {
+          const ColConst cc = col_const<BF16, WK>(p, nn, col_ok);
+          escale = (WK == kWFp8 || cc.fast) ? cc.s : 1.f;
+        }
+        if (p.bias && col_ok) bias_v = act_f32(p.bias[nn], BF16);
+      }
+      float* part = (it.slot >= 0)
+                        ? p.partial + (static_cast<int64_t>(it.tile) * p.max_slots + it.slot) * (BN * kWqNBlock)
+                        : nullptr;
+      constexpr int kChunk = 16;  // accumulator columns (m rows) per tcgen05.ld
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += kChunk) {
-        uint32_t v[32];
-        if constexpr (kChunk == 32)
-          tmem_ld_x32(tmem + lane_addr + kAccCol + c0, v);
-        else
-          tmem_ld_x16(tmem + lane_addr + kAccCol + c0, v);
+        uint32_t v[kChunk];
+        tmem_ld_x16(tmem + lane_addr + ab * C::kAccCols + c0, v);
         tmem_wait_ld();
-        if (col_ok) {
+        if (part) {
 #pragma unroll
-          for (int j = 0; j < kChunk; ++j) {
-            const int64_t mm = m0 + c0 + j;
+          for (int q = 0; q < kChunk; ++q) part[(c0 + q) * kWqNBlock + nl] = __uint_as_float(v[q]);
+        } else if (col_ok) {
+#pragma unroll
+          for (int q = 0; q < kChunk; ++q) {
+            const int64_t mm = m0 + c0 + q;
             if (mm < p.m) {
-              const float acc = __uint_as_float(v[j]);
-              if (p.splits == 1) {
-                float y = acc * escale + bias_v;
-                if (p.x3) y += act_f32(p.x3[mm * p.n + nn], BF16);
-                p.out[mm * p.n + nn] = f32_act(y, BF16);
-              } else {
-                p.partial[(static_cast<int64_t>(split) * p.m + mm) * p.n + nn] = acc;
-              }
+              float y = __uint_as_float(v[q]) * escale + bias_v;
+              if (p.x3) y += act_f32(p.x3[mm * p.n + nn], BF16);
+              p.out[mm * p.n + nn] = f32_act(y, BF16);
             }
           }
         }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar_accempty[ab]);
+      ++j;
+    }
+  } else {
+    // ============================================================ dequantisation
+    const int dg = (warp - 7) >> 2;               // group: takes k steps g with g % DG == dg
+    const int quad = warp & 3;                    // TMEM lane quadrant this warp may access
+    const int r = quad * 32 + lane;               // weight column within the 128-column block
+    const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+    const bool grp = (p.mode == kPerGroup);
+    const int gq = grp ? p.group_size / 32 : 1;   // 32-wide halves per group
+    uint32_t g = 0;
+    bool live = true;
+    while (live && walk.next(p, it)) {
+      const int nb = it.tile % p.num_nb;
+      const int nn = nb * kWqNBlock + r;
+      const bool col_ok = nn < p.n;
+      ColConst cc{};
+      if (!grp) cc = col_const<BF16, WK>(p, nn, col_ok);
+      // per-group scale/offset come straight from global memory (L2), one of
+      // this group's k steps ahead of their use
+      const int kt_first = it.kt0 + static_cast<int>((dg - static_cast<int>(g % DG) + DG) % DG);
+      GroupRow grow{};
+      GroupSO so_next{};
+      if (grp && kt_first < it.kt1) {
+        grow.init(2 * kt_first, gq);
+        so_next = load_group_so(p, kt_first, grow, gq, nn, col_ok);
+      }
+      for (int kt = it.kt0; kt < it.kt1; ++kt, ++g) {
+        if (static_cast<int>(g % DG) != dg) continue;
+        const GroupSO so = so_next;
+        if (grp && kt + DG < it.kt1) {
+          grow.advance(2 * DG, gq);
+          so_next = load_group_so(p, kt + DG, grow, gq, nn, col_ok);
+        }
+        const int sw = g % SW;
+        const int as = g % AS;
+        // 1) weight tile -> registers, then hand the stage back to the producer
+        bool got = mbar_wait(&bar_wfull[sw], (g / SW) & 1, abort_flag, p.err, kDevTimeoutDequant);
+        if (!__all_sync(kFull, got)) {
+          live = false;
+          break;
+        }
+        const uint8_t* wt = s_w + sw * kTile;
+        constexpr int kChunks = (WK == kW4) ? 2 : 4;
+        uint4 ch[kChunks];
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) ch[c] = *reinterpret_cast<const uint4*>(wt + (c * kWqNBlock + r) * 16);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_wempty[sw]);
+        // 2) dequantise into an A stage of TMEM
+        got = mbar_wait(&bar_aempty[as], ((g / AS) & 1) ^ 1, abort_flag, p.err, kDevTimeoutDequant);
+        if (!__all_sync(kFull, got)) {  // tcgen05.st below is warp-collective
+          live = false;
+          break;
+        }
+        uint32_t a[32];
+        if constexpr (WK == kW4) {
+          if (grp) {
+            dq4_group_half<BF16, 0>(ch[0], so.s[0], so.o[0], a);
+            dq4_group_half<BF16, 1>(ch[1], so.s[1], so.o[1], a);
+          } else if (cc.fast) {
+            dq4_fast<BF16, false>(ch[0], cc.c2, 0u, a);
+            dq4_fast<BF16, false>(ch[1], cc.c2, 0u, a + 16);
+          } else {
+            dq4_general<BF16>(ch[0], cc.off, cc.s, a);
+            dq4_general<BF16>(ch[1], cc.off, cc.s, a + 16);
+          }
+        } else if constexpr (WK == kW8) {
+          if (grp) {
+            dq8_group_half<BF16, 0>(ch[0], ch[1], so.s[0], so.o[0], a);
+            dq8_group_half<BF16, 1>(ch[2], ch[3], so.s[1], so.o[1], a);
+          } else if (cc.fast) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) dq8_fast<BF16, false>(ch[c], cc.off, cc.s, cc.c2, 0u, a + 8 * c);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) dq8_general<BF16>(ch[c], cc.off, cc.s, a + 8 * c);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) dq_fp8<BF16>(ch[c], a + 8 * c);
+        }
+        tmem_st_x32(tmem + lane_addr + C::kACol0 + as * 32, a);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_afull[as]);
       }
     }
   }
@@ -466,37 +643,100 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int BN, int WK, bool BF16>
-cudaError_t launch_one(const CUtensorMap& tmap, const WqParams& p, cudaStream_t s) {
-  constexpr int smem = Cfg<BN>::template smem_bytes<WK>();
-  auto kern = wqmm_tc_kernel<BN, WK, BF16>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+template <int BN, int DG, int WK, bool BF16>
+cudaError_t launch_one(const CUtensorMap& tmap, const WqParams& p, int grid, cudaStream_t s) {
+  using C = Cfg<BN, DG, WK>;
+  auto kern = wqmm_tc_kernel<BN, DG, WK, BF16>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int64_t grid = static_cast<int64_t>(p.num_mb) * p.num_nb * p.splits;
-  if (grid <= 0 || grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
-  kern<<<static_cast<unsigned>(grid), kThreads, smem, s>>>(tmap, p);
+  if (grid <= 0) return cudaErrorInvalidConfiguration;
+  kern<<<static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, s>>>(tmap, p);
   return cudaGetLastError();
 }
 
+// dequantisation groups: small tiles have little MMA work per k step, so more
+// k steps must be dequantised at once to keep the weight stream flowing
 template <int BN>
-cudaError_t launch_bn(const CUtensorMap& tmap, const WqParams& p, int wk, bool bf16, cudaStream_t s) {
-  if (wk == kW4) return bf16 ? launch_one<BN, kW4, true>(tmap, p, s) : launch_one<BN, kW4, false>(tmap, p, s);
-  if (wk == kW8) return bf16 ? launch_one<BN, kW8, true>(tmap, p, s) : launch_one<BN, kW8, false>(tmap, p, s);
-  return bf16 ? launch_one<BN, kWFp8, true>(tmap, p, s) : launch_one<BN, kWFp8, false>(tmap, p, s);
+constexpr int dgroups() {
+  return 4;
+}
+
+template <int BN>
+cudaError_t launch_bn(const CUtensorMap& tmap, const WqParams& p, int wk, bool bf16, int grid, cudaStream_t s) {
+  constexpr int DG = dgroups<BN>();
+  if (wk == kW4)
+    return bf16 ? launch_one<BN, DG, kW4, true>(tmap, p, grid, s) : launch_one<BN, DG, kW4, false>(tmap, p, grid, s);
+  if (wk == kW8)
+    return bf16 ? launch_one<BN, DG, kW8, true>(tmap, p, grid, s) : launch_one<BN, DG, kW8, false>(tmap, p, grid, s);
+  return bf16 ? launch_one<BN, DG, kWFp8, true>(tmap, p, grid, s)
+              : launch_one<BN, DG, kWFp8, false>(tmap, p, grid, s);
+}
+
+// ---------------------------------------------------------------- stream-K fix-up
+// out = (sum of the tile's partials, in slot order) * epilogue scale + bias + x3.
+// One 128-thread block row per (tile, m row); warp = 32 aligned columns, the
+// same grouping the GEMM's epilogue uses for its warp-uniform scale choice.
+__global__ void __launch_bounds__(128) wqmm_fixup_kernel(const FixupParams p) {
+  const int64_t rows = static_cast<int64_t>(p.num_tiles) * p.bn;
+  const int64_t T = static_cast<int64_t>(p.num_tiles) * p.kt_total;
+  const int nl = threadIdx.x;  // column within the 128-column block
+  const bool bf16 = p.act_bf16 != 0;
+  for (int64_t rr = blockIdx.x; rr < rows; rr += gridDim.x) {
+    const int tile = static_cast<int>(rr / p.bn);
+    const int ml = static_cast<int>(rr % p.bn);
+    const int nb = tile % p.num_nb;
+    const int64_t mm = static_cast<int64_t>(tile / p.num_nb) * p.bn + ml;
+    const int nn = nb * kWqNBlock + nl;
+    const bool col_ok = nn < p.n;
+    const int64_t first = static_cast<int64_t>(tile) * p.kt_total;
+    const int slots = static_cast<int>(sk_owner(first + p.kt_total - 1, T, p.grid) - sk_owner(first, T, p.grid)) + 1;
+    float acc = 0.f;
+    for (int s = 0; s < slots; ++s)
+      acc += p.partial[((static_cast<int64_t>(tile) * p.max_slots + s) * p.bn + ml) * kWqNBlock + nl];
+    float escale = 1.f;
+    if (p.mode != kPerGroup) {
+      const int idx = (p.mode == kPerTensor) ? 0 : (col_ok ? nn : 0);
+      const float off = p.offset ? act_f32(p.offset[idx], bf16) : 0.f;
+      const bool fast = __all_sync(kFull, small_int(off));
+      if (fast) escale = act_f32(p.scale[idx], bf16);
+    }
+    if (col_ok && mm < p.m) {
+      float y = acc * escale;
+      if (p.bias) y += act_f32(p.bias[nn], bf16);
+      if (p.x3) y += act_f32(p.x3[mm * p.n + nn], bf16);
+      p.out[mm * p.n + nn] = f32_act(y, bf16);
+    }
+  }
 }
 
 }  // namespace
 
+int wqmm_ctas_per_sm(int bn, int wk) {
+  (void)bn;
+  (void)wk;
+  return 1;  // every configuration uses most of the SM's shared memory for its ring
+}
+
 cudaError_t launch_wqmm_gemm(const CUtensorMap& tmap_x1, const WqParams& p, int bn, int wk, bool act_bf16,
-                             cudaStream_t s) {
+                             int grid, cudaStream_t s) {
   switch (bn) {
-    case 16: return launch_bn<16>(tmap_x1, p, wk, act_bf16, s);
-    case 32: return launch_bn<32>(tmap_x1, p, wk, act_bf16, s);
-    case 64: return launch_bn<64>(tmap_x1, p, wk, act_bf16, s);
-    case 128: return launch_bn<128>(tmap_x1, p, wk, act_bf16, s);
-    case 256: return launch_bn<256>(tmap_x1, p, wk, act_bf16, s);
+    case 16: return launch_bn<16>(tmap_x1, p, wk, act_bf16, grid, s);
+    case 32: return launch_bn<32>(tmap_x1, p, wk, act_bf16, grid, s);
+    case 64: return launch_bn<64>(tmap_x1, p, wk, act_bf16, grid, s);
+    case 128: return launch_bn<128>(tmap_x1, p, wk, act_bf16, grid, s);
+    case 192: return launch_bn<192>(tmap_x1, p, wk, act_bf16, grid, s);
+    case 256: return launch_bn<256>(tmap_x1, p, wk, act_bf16, grid, s);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_wqmm_fixup(const FixupParams& p, cudaStream_t s) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t rows = static_cast<int64_t>(p.num_tiles) * p.bn;
+  const int64_t cap = static_cast<int64_t>(sms) * 16;
+  wqmm_fixup_kernel<<<static_cast<unsigned>(rows < cap ? rows : cap), 128, 0, s>>>(p);
+  return cudaGetLastError();
 }
 
 }  // namespace wqmm
