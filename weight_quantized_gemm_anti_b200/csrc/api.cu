@@ -408,8 +408,8 @@ extern "C" wqmm_status wqmm_get_workspace_size(const wqmm_tensor* x1, const wqmm
     const char* sk_env = std::getenv("WQMM_STREAMK");
     const bool force_sk = sk_env && std::atoi(sk_env) == 1;
     const bool forbid_sk = sk_env && std::atoi(sk_env) == 0;
-    if (!forbid_sk && (force_sk || tiles < 2 * slots) && kt >= 2) {
-      // few tiles: spread all k steps evenly over one CTA per SM
+    if (!forbid_sk && (force_sk || tiles < slots) && kt >= 2) {
+      // fewer tiles than SMs: spread all k steps evenly over one CTA per SM
       ex->stream_k = 1;
       const int64_t total = tiles * kt;
       ex->grid = static_cast<int>(total < slots ? total : slots);

@@ -53,6 +53,7 @@ namespace wqmm {
 namespace {
 
 constexpr unsigned kFull = 0xFFFFFFFFu;
+constexpr int kProducerLanes = 4;
 
 constexpr int pow2ceil(int v) { return v <= 32 ? 32 : v <= 64 ? 64 : v <= 128 ? 128 : v <= 256 ? 256 : 512; }
 constexpr int cmin(int a, int b) { return a < b ? a : b; }
@@ -66,20 +67,26 @@ struct Cfg {
   static constexpr int kAccCols = BN < 32 ? 32 : BN;
   static constexpr int kNAcc = (2 * kAccCols + 4 * 32 <= 512) ? 2 : 1;
   static constexpr int kACol0 = kNAcc * kAccCols;
-  // TMEM A stages: as many as fit (up to 8), a multiple of DG so that every
+  // TMEM A stages: as many as fit (up to 12), a multiple of DG so that every
   // dequantisation group owns its own stages
-  static constexpr int kAStages = cmin(8, (512 - kACol0) / 32 / DG * DG);
+  static constexpr int kAStages = cmin(12, (512 - kACol0) / 32 / DG * DG);
   static constexpr int kTmemCols = pow2ceil(kACol0 + kAStages * 32);
   // shared memory: an x1 ring (read by the MMA) and a weight ring (read by the
   // dequantisers, released as soon as a tile is in registers)
   static constexpr int kSmemBudget = 200 * 1024;
   static constexpr int kXStages = cmin(16, cmax(4, (kSmemBudget * 3 / 5) / kX1Bytes));
   static constexpr int kWStages = cmin(32, (kSmemBudget - kXStages * kX1Bytes) / kTile);
+  // The MMA issuer waits once per batch of k steps (half the A stages) and then
+  // issues the whole batch: every barrier wait in the issuing thread costs the
+  // tensor pipe its queued overlap, so a wait has to be followed by roughly
+  // 800+ cycles of MMA work to keep the pipe busy.
+  static constexpr int kBatch = cmax(1, cmin(kAStages / 2, kXStages / 2));
   static constexpr int kThreads = 32 * (7 + 4 * DG);
   static constexpr int kSmemBytes = kXStages * kX1Bytes + kWStages * kTile + 1024;
   static_assert(kAStages >= DG && kAStages % DG == 0, "A stages");
   static_assert(kACol0 + kAStages * 32 <= 512, "TMEM budget");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+  static_assert(kXStages >= 2 * kBatch && kAStages >= 2 * kBatch, "a batch must fit twice in each ring");
 };
 
 __device__ __forceinline__ float act_f32(uint16_t v, bool bf16) {
@@ -362,6 +369,10 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
   constexpr int SX = C::kXStages;
   constexpr int SW = C::kWStages;
   constexpr int AS = C::kAStages;
+  // Completion of k step g is one commit on bar_done[g % RD] (phase g / RD).  A
+  // waiter for step g - SX (x1 producer) or g - AS (dequantiser) can never see
+  // that barrier lapped, since step g - X + RD needs data it has not yet made.
+  constexpr int RD = SX + AS;
   constexpr int kTile = C::kTile;
   constexpr uint32_t kIdesc = idesc_make(1u, BF16 ? 1u : 0u, 128u, static_cast<uint32_t>(BN));
 
@@ -371,11 +382,10 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
   uint8_t* s_w = s_x1 + SX * C::kX1Bytes;  // SW x packed weight tile
 
   __shared__ __align__(8) uint64_t bar_xfull[SX];
-  __shared__ __align__(8) uint64_t bar_xempty[SX];
+  __shared__ __align__(8) uint64_t bar_done[RD];  // one commit per k step: x1 slab and A stage free
   __shared__ __align__(8) uint64_t bar_wfull[SW];
   __shared__ __align__(8) uint64_t bar_wempty[SW];
   __shared__ __align__(8) uint64_t bar_afull[AS];
-  __shared__ __align__(8) uint64_t bar_aempty[AS];
   __shared__ __align__(8) uint64_t bar_accfull[2];
   __shared__ __align__(8) uint64_t bar_accempty[2];
   __shared__ __align__(8) uint64_t bar_drain;
@@ -388,7 +398,6 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < SX; ++i) {
       mbar_init(&bar_xfull[i], 1);
-      mbar_init(&bar_xempty[i], 1);
     }
     for (int i = 0; i < SW; ++i) {
       mbar_init(&bar_wfull[i], 1);
@@ -396,8 +405,8 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
     }
     for (int i = 0; i < AS; ++i) {
       mbar_init(&bar_afull[i], 4);
-      mbar_init(&bar_aempty[i], 1);
     }
+    for (int i = 0; i < RD; ++i) mbar_init(&bar_done[i], 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_accfull[i], 1);
       mbar_init(&bar_accempty[i], 4);
@@ -424,20 +433,28 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
     // ============================================================ producers
     // warp 0: x1 tiles (one 2-D tensor copy per k step) for the MMA;
     // warp 6: packed weight tiles (one 1-D bulk copy per k step) for the dequantisers.
-    if (lane == 0) {
+    // A copy instruction occupies its issuing thread for hundreds of cycles
+    // whatever its size, so kProducerLanes lanes issue alternate k steps.
+    if (lane < kProducerLanes) {
       const bool is_x = (warp == 0);
-      if (is_x) prefetch_tensormap(&tmap_x1);
+      if (is_x && lane == 0) prefetch_tensormap(&tmap_x1);
       const int ns = is_x ? SX : SW;
       uint64_t* full = is_x ? bar_xfull : bar_wfull;
-      uint64_t* empty = is_x ? bar_xempty : bar_wempty;
       uint32_t g = 0;
       bool live = true;
       while (live && walk.next(p, it)) {
         const int nb = it.tile % p.num_nb;
         const int32_t m0 = static_cast<int32_t>(static_cast<int64_t>(it.tile / p.num_nb) * BN);
         for (int kt = it.kt0; kt < it.kt1; ++kt, ++g) {
+          if (static_cast<int>(g % kProducerLanes) != lane) continue;
           const int st = g % ns;
-          if (!mbar_wait(&empty[st], ((g / ns) & 1) ^ 1, abort_flag, p.err, kDevTimeoutProducer)) {
+          // x1 slab free once the MMA of step g - SX is done; weight stage once read
+          const bool ok = is_x ? (g < static_cast<uint32_t>(SX) ||
+                                  mbar_wait_sleep(&bar_done[(g - SX) % RD], ((g - SX) / RD) & 1, abort_flag,
+                                                  p.err, kDevTimeoutProducer, 32, 256))
+                               : mbar_wait_sleep(&bar_wempty[st], ((g / ns) & 1) ^ 1, abort_flag, p.err,
+                                                 kDevTimeoutProducer, 32, 256);
+          if (!ok) {
             live = false;
             break;
           }
@@ -451,9 +468,10 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
           }
         }
       }
-      // every copy issued into the ring has landed before the CTA may exit
+      // every copy this lane issued into the ring has landed before the CTA may exit
       const uint32_t first = g > static_cast<uint32_t>(ns) ? g - ns : 0;
       for (uint32_t i = first; i < g; ++i) {
+        if (static_cast<int>(i % kProducerLanes) != lane) continue;
         volatile int no_abort = 0;
         mbar_wait(&full[i % ns], (i / ns) & 1, &no_abort, p.err, kDevTimeoutDrain);
       }
@@ -468,23 +486,30 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
         if (!mbar_wait(&bar_accempty[ab], ((j / C::kNAcc) & 1) ^ 1, abort_flag, p.err, kDevTimeoutMma)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + ab * C::kAccCols;
-        for (int kt = it.kt0; kt < it.kt1; ++kt, ++g) {
-          const int sx = g % SX;
-          const int as = g % AS;
-          if (!mbar_wait(&bar_xfull[sx], (g / SX) & 1, abort_flag, p.err, kDevTimeoutMma) ||
-              !mbar_wait(&bar_afull[as], (g / AS) & 1, abort_flag, p.err, kDevTimeoutMma)) {
-            live = false;
-            break;
+        for (int kt = it.kt0; kt < it.kt1 && live;) {
+          const int nbs = min(C::kBatch, it.kt1 - kt);
+          // wait for every x1 slab and A stage of the batch, then issue it whole
+          // afull of a step implies its x1 slab has landed (the dequantisers check)
+          for (int jj = 0; jj < nbs && live; ++jj) {
+            const uint32_t gg = g + jj;
+            live = mbar_wait(&bar_afull[gg % AS], (gg / AS) & 1, abort_flag, p.err, kDevTimeoutMma);
           }
+          if (!live) break;
           tc_fence_after();
-          const uint32_t b_base = smem_u32(s_x1 + sx * C::kX1Bytes);
+          for (int jj = 0; jj < nbs; ++jj) {
+            const uint32_t gg = g + jj;
+            const int sx = gg % SX;
+            const int as = gg % AS;
+            const uint32_t b_base = smem_u32(s_x1 + sx * C::kX1Bytes);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            mma_f16_ts(d_tmem, tmem + C::kACol0 + as * 32 + kk * 8, sdesc_kmajor_sw128(b_base + kk * 32), kIdesc,
-                       (kt > it.kt0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {
+              mma_f16_ts(d_tmem, tmem + C::kACol0 + as * 32 + kk * 8, sdesc_kmajor_sw128(b_base + kk * 32), kIdesc,
+                         (kt + jj > it.kt0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(&bar_done[gg % RD]);
           }
-          mma_commit(&bar_xempty[sx]);
-          mma_commit(&bar_aempty[as]);
+          kt += nbs;
+          g += nbs;
         }
         if (!live) break;
         mma_commit(&bar_accfull[ab]);
@@ -501,7 +526,8 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
     uint32_t j = 0;
     while (walk.next(p, it)) {
       const int ab = j % C::kNAcc;
-      bool ready = mbar_wait(&bar_accfull[ab], (j / C::kNAcc) & 1, abort_flag, p.err, kDevTimeoutEpilogue);
+      bool ready =
+          mbar_wait_sleep(&bar_accfull[ab], (j / C::kNAcc) & 1, abort_flag, p.err, kDevTimeoutEpilogue, 256, 2048);
       if (!__all_sync(kFull, ready && !*abort_flag)) break;
       tc_fence_after();
       const int nb = it.tile % p.num_nb;
@@ -581,7 +607,7 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
         const int sw = g % SW;
         const int as = g % AS;
         // 1) weight tile -> registers, then hand the stage back to the producer
-        bool got = mbar_wait(&bar_wfull[sw], (g / SW) & 1, abort_flag, p.err, kDevTimeoutDequant);
+        bool got = mbar_wait_sleep(&bar_wfull[sw], (g / SW) & 1, abort_flag, p.err, kDevTimeoutDequant, 32, 256);
         if (!__all_sync(kFull, got)) {
           live = false;
           break;
@@ -594,7 +620,10 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar_wempty[sw]);
         // 2) dequantise into an A stage of TMEM
-        got = mbar_wait(&bar_aempty[as], ((g / AS) & 1) ^ 1, abort_flag, p.err, kDevTimeoutDequant);
+        got = mbar_wait_sleep(&bar_xfull[g % SX], (g / SX) & 1, abort_flag, p.err, kDevTimeoutDequant, 32, 256);
+        if (got && g >= static_cast<uint32_t>(AS))
+          got = mbar_wait_sleep(&bar_done[(g - AS) % RD], ((g - AS) / RD) & 1, abort_flag, p.err,
+                                kDevTimeoutDequant, 32, 256);
         if (!__all_sync(kFull, got)) {  // tcgen05.st below is warp-collective
           live = false;
           break;

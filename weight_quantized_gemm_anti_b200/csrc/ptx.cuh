@@ -93,6 +93,30 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Bounded wait that yields the issue slots while it waits: after a few polls it
+// sleeps with exponential backoff (from min_ns up to max_ns).  For roles whose
+// waits are long or off the critical path, so that spinning warps do not take
+// issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                uint32_t* err_word, uint32_t code, uint32_t min_ns,
+                                                uint32_t max_ns) {
+  for (int i = 0; i < 4; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  uint32_t ns = min_ns;
+  while (true) {
+    __nanosleep(ns);
+    if (mbar_try_wait(bar, parity)) return true;
+    ns = ns * 2 > max_ns ? max_ns : ns * 2;
+    if (*abort) return false;
+    if (globaltimer() - t0 > WQMM_WAIT_NS) {
+      *abort = 1;
+      if (err_word) atomicCAS(err_word, 0u, code);
+      return false;
+    }
+  }
+}
+
 // ------------------------------------------------------------------ async proxy fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
