@@ -182,6 +182,30 @@ WQMM_API wqmm_status qmm_run(void* workspace, uint64_t workspace_size, wqmm_exec
 WQMM_API wqmm_status wqmm_pack_weight_size(const wqmm_tensor* x2, int32_t for_int8_gemm, uint64_t* packed_bytes);
 WQMM_API wqmm_status wqmm_pack_weight(const wqmm_tensor* x2, int32_t for_int8_gemm, void* packed, wqmm_stream stream);
 
+/* ================================================================ no-allocation variant
+ *
+ * wqmm_matmul_no_alloc -- both phases of the anti-quant GEMM in one call, for
+ * callers that cannot allocate device memory (a region being captured into a
+ * CUDA graph, a component with a fixed memory budget, a foreign ABI that passes
+ * tensors but no allocator).  The operator pages have no counterpart: it exists
+ * for this library's callers only.  Arguments are those of
+ * wqmm_get_workspace_size minus the workspace outputs, plus the stream.
+ *
+ * The workspace is a fixed 16 MiB array in device memory owned by the library
+ * (every GPU that loads the library keeps it until the process exits).
+ * Problems that need more are rejected with WQMM_ERR_WORKSPACE before any
+ * launch; pre-packing the weight keeps the need small.  No device memory is
+ * allocated or freed.  All calls on a device share the array: calls that
+ * overlap on the GPU race, so serialise them.  The first call on a device
+ * looks up the array's address (with that device current); make it before any
+ * stream capture begins.
+ */
+WQMM_API wqmm_status wqmm_matmul_no_alloc(const wqmm_tensor* x1, const wqmm_tensor* x2, const wqmm_tensor* bias,
+                                          const wqmm_tensor* antiquant_scale, const wqmm_tensor* antiquant_offset,
+                                          const wqmm_tensor* x3, const char* group, const char* reduce_op,
+                                          int64_t comm_turn, int64_t stream_mode, int64_t antiquant_group_size,
+                                          const wqmm_tensor* output, wqmm_stream stream);
+
 /* ================================================================ utilities */
 
 /* Release an executor that was never passed to a *_run call (NULL is ignored). */

@@ -217,6 +217,23 @@ def qmm_debug_set_raw_accumulator(executor, acc_ptr: int) -> int:
     return lib().qmm_debug_set_raw_accumulator(executor, acc_ptr)
 
 
+def wqmm_matmul_no_alloc(x1, x2, bias, antiquant_scale, antiquant_offset, x3, group, reduce_op, comm_turn,
+                         stream_mode, antiquant_group_size, output, stream=None) -> int:
+    """Both phases of the anti-quant GEMM in one call, with the library's fixed
+    16 MiB device workspace instead of a caller-provided one (for callers that
+    cannot allocate device memory).  Returns the C status."""
+    L = lib()
+    f = L.wqmm_matmul_no_alloc
+    if f.argtypes is None:
+        T = ctypes.POINTER(WqmmTensor)
+        f.argtypes = [T, T, T, T, T, T, ctypes.c_char_p, ctypes.c_char_p, ctypes.c_int64, ctypes.c_int64,
+                      ctypes.c_int64, T, ctypes.c_void_p]
+        f.restype = ctypes.c_int32
+    return f(_ref(x1), _ref(x2), _ref(bias), _ref(antiquant_scale), _ref(antiquant_offset), _ref(x3),
+             None if group is None else group.encode(), None if reduce_op is None else reduce_op.encode(),
+             int(comm_turn), int(stream_mode), int(antiquant_group_size), _ref(output), _stream_handle(stream))
+
+
 def check(status: int) -> None:
     if status != SUCCESS:
         raise WqmmError(status, wqmm_last_error())

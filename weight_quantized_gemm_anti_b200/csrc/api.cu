@@ -882,3 +882,8 @@ extern "C" wqmm_status wqmm_device_error(uint32_t* code, int32_t reset) {
   }
   return ok();
 }
+
+namespace wqmm {
+// Record a message for wqmm_last_error() from another translation unit of the library.
+wqmm_status report_error(wqmm_status code, const char* msg) { return fail(code, "%s", msg); }
+}  // namespace wqmm

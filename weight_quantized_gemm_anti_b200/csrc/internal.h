@@ -130,4 +130,7 @@ cudaError_t launch_qmm_gemm(const CUtensorMap& tmap_x1, const QParams& p, cudaSt
 // Device error word of the library (first kernel error code, 0 if none).
 uint32_t* device_error_word();
 
+// Set the calling thread's wqmm_last_error() message and return `code`.
+int32_t report_error(int32_t code, const char* msg);
+
 }  // namespace wqmm
