@@ -272,6 +272,23 @@ def cpu_baseline(name: str, rows: int):
             "sample": f"{len(r)} of {case.m} output rows x all {case.n} columns of {name} ({dt:.1f} s)"}
 
 
+def max_over_ranks(values, device):
+    """Elementwise max of per-rank values over the process group (identity for one rank).
+    Every rank must call it, in the same order."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def replica_throughput(flops_per_step: float, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job TFLOP/s of `world` independent replicas that each ran `steps`
+    steps, timed by the slowest rank (max_ms, device time)."""
+    return flops_per_step * world * steps / (max_ms * 1e-3) / 1e12
+
+
 def gpu_arm(args):
     import torch
     import torch.distributed as dist
@@ -301,19 +318,13 @@ def gpu_arm(args):
     if world > 1:
         dist.barrier()
     clocks = sampler.stop(local) if rank == 0 else None
-    total_ms = sum(times)
-    t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = max_over_ranks([sum(times)], "cuda")[0]
     st, code = W.wqmm_device_error(reset=True)
     if st != 0 or code != 0:
         raise RuntimeError(f"device error word {code}")
 
     e2e_ms, h2d, d2h = time_e2e(prob, max(3, min(args.steps, 20)), 2)
-    e2e_t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+    e2e_ms = max_over_ranks([e2e_ms], "cuda")[0]
 
     extra = {}
     if rank == 0 and world == 1 and not args.no_extra:
@@ -341,8 +352,7 @@ def gpu_arm(args):
 
     if rank == 0:
         ms_step = max_ms / args.steps
-        flops_all = prob.flops * world * args.steps
-        value = flops_all / (max_ms * 1e-3) / 1e12
+        value = replica_throughput(prob.flops, world, args.steps, max_ms)
         achieved = prob.flops / (ms_step * 1e-3) / 1e12
         peak = peaks["bf16_tflops"]
         traffic = load_traffic(args.config)
@@ -353,7 +363,7 @@ def gpu_arm(args):
             "config": {"workload": args.config, "m": prob.case.m, "k": prob.case.k, "n": prob.case.n,
                        "weight": "int4 packed, per-group g=128 scale+offset", "l2": "flushed before every step "
                        "(512 MB write outside the timed interval)", "parallelism": f"replicas x{world}"},
-            "e2e": {"value": round(prob.flops * world / (float(e2e_t.item()) * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "e2e": {"value": round(replica_throughput(prob.flops, world, 1, e2e_ms), 3), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": prob.launches_per_step() * args.steps,
             "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
