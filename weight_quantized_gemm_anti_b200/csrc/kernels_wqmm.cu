@@ -53,7 +53,6 @@ namespace wqmm {
 namespace {
 
 constexpr unsigned kFull = 0xFFFFFFFFu;
-constexpr int kProducerLanes = 4;
 
 constexpr int pow2ceil(int v) { return v <= 32 ? 32 : v <= 64 ? 64 : v <= 128 ? 128 : v <= 256 ? 256 : 512; }
 constexpr int cmin(int a, int b) { return a < b ? a : b; }
@@ -71,18 +70,27 @@ struct Cfg {
   // dequantisation group owns its own stages
   static constexpr int kAStages = cmin(12, (512 - kACol0) / 32 / DG * DG);
   static constexpr int kTmemCols = pow2ceil(kACol0 + kAStages * 32);
-  // shared memory: an x1 ring (read by the MMA) and a weight ring (read by the
-  // dequantisers, released as soon as a tile is in registers)
-  static constexpr int kSmemBudget = 200 * 1024;
-  static constexpr int kXStages = cmin(16, cmax(4, (kSmemBudget * 3 / 5) / kX1Bytes));
-  static constexpr int kWStages = cmin(32, (kSmemBudget - kXStages * kX1Bytes) / kTile);
+  // shared memory: a weight ring (read by the dequantisers, released as soon
+  // as a tile is in registers) and an x1 ring (read by the MMA).  An x1 slab is
+  // refilled only after the MMA of the step SX earlier has finished, so SX - 1
+  // steps of MMA work have to cover the latency of its tensor copy: for wide m
+  // tiles the x1 ring gets the depth and 40-48 KB of weights cover theirs.
+  // Narrow m tiles stream weights from HBM: the weight ring then takes most of
+  // the space, to keep enough bytes in flight.
+  // epilogue staging: kEpiRows output rows x 128 columns, fp32
+  static constexpr int kEpiRows = 16;
+  static constexpr int kStageBytes = kEpiRows * 128 * 4;
+  static constexpr int kSmemBudget = 224 * 1024 - kStageBytes;
+  static constexpr int kWStages =
+      BN <= 64 ? cmin(32, (kSmemBudget - 8 * kX1Bytes) / kTile) : ((WK == kW4) ? 10 : 6);
+  static constexpr int kXStages = cmin(16, (kSmemBudget - kWStages * kTile) / kX1Bytes);
   // The MMA issuer waits once per batch of k steps (half the A stages) and then
   // issues the whole batch: every barrier wait in the issuing thread costs the
   // tensor pipe its queued overlap, so a wait has to be followed by roughly
   // 800+ cycles of MMA work to keep the pipe busy.
   static constexpr int kBatch = cmax(1, cmin(kAStages / 2, kXStages / 2));
   static constexpr int kThreads = 32 * (7 + 4 * DG);
-  static constexpr int kSmemBytes = kXStages * kX1Bytes + kWStages * kTile + 1024;
+  static constexpr int kSmemBytes = kXStages * kX1Bytes + kWStages * kTile + kStageBytes + 1024;
   static_assert(kAStages >= DG && kAStages % DG == 0, "A stages");
   static_assert(kACol0 + kAStages * 32 <= 512, "TMEM budget");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -380,6 +388,7 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* s_x1 = smem;                  // SX x (BN x 128 B), 1024-aligned slabs
   uint8_t* s_w = s_x1 + SX * C::kX1Bytes;  // SW x packed weight tile
+  uint8_t* s_stage = s_w + SW * kTile;     // epilogue staging tile (fp32)
 
   __shared__ __align__(8) uint64_t bar_xfull[SX];
   __shared__ __align__(8) uint64_t bar_done[RD];  // one commit per k step: x1 slab and A stage free
@@ -433,31 +442,31 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
     // ============================================================ producers
     // warp 0: x1 tiles (one 2-D tensor copy per k step) for the MMA;
     // warp 6: packed weight tiles (one 1-D bulk copy per k step) for the dequantisers.
-    // A copy instruction occupies its issuing thread for hundreds of cycles
-    // whatever its size, so kProducerLanes lanes issue alternate k steps.
-    if (lane < kProducerLanes) {
-      const bool is_x = (warp == 0);
-      if (is_x && lane == 0) prefetch_tensormap(&tmap_x1);
-      const int ns = is_x ? SX : SW;
-      uint64_t* full = is_x ? bar_xfull : bar_wfull;
-      uint32_t g = 0;
-      bool live = true;
-      while (live && walk.next(p, it)) {
-        const int nb = it.tile % p.num_nb;
-        const int32_t m0 = static_cast<int32_t>(static_cast<int64_t>(it.tile / p.num_nb) * BN);
-        for (int kt = it.kt0; kt < it.kt1; ++kt, ++g) {
-          if (static_cast<int>(g % kProducerLanes) != lane) continue;
-          const int st = g % ns;
-          // x1 slab free once the MMA of step g - SX is done; weight stage once read
-          const bool ok = is_x ? (g < static_cast<uint32_t>(SX) ||
-                                  mbar_wait_sleep(&bar_done[(g - SX) % RD], ((g - SX) / RD) & 1, abort_flag,
-                                                  p.err, kDevTimeoutProducer, 32, 256))
-                               : mbar_wait_sleep(&bar_wempty[st], ((g / ns) & 1) ^ 1, abort_flag, p.err,
-                                                 kDevTimeoutProducer, 32, 256);
-          if (!ok) {
-            live = false;
-            break;
-          }
+    // The whole warp walks the ring and waits; one elected lane issues each
+    // copy, so its operands are warp-uniform.
+    const bool is_x = (warp == 0);
+    if (is_x && elect_one()) prefetch_tensormap(&tmap_x1);
+    __syncwarp();
+    const int ns = is_x ? SX : SW;
+    uint64_t* full = is_x ? bar_xfull : bar_wfull;
+    uint32_t g = 0;
+    bool live = true;
+    while (live && walk.next(p, it)) {
+      const int nb = it.tile % p.num_nb;
+      const int32_t m0 = static_cast<int32_t>(static_cast<int64_t>(it.tile / p.num_nb) * BN);
+      for (int kt = it.kt0; kt < it.kt1; ++kt, ++g) {
+        const int st = g % ns;
+        // x1 slab free once the MMA of step g - SX is done; weight stage once read
+        const bool ok = is_x ? (g < static_cast<uint32_t>(SX) ||
+                                mbar_wait(&bar_done[(g - SX) % RD], ((g - SX) / RD) & 1, abort_flag, p.err,
+                                          kDevTimeoutProducer))
+                             : mbar_wait_sleep(&bar_wempty[st], ((g / ns) & 1) ^ 1, abort_flag, p.err,
+                                               kDevTimeoutProducer, 32, 256);
+        if (!__all_sync(kFull, ok)) {
+          live = false;
+          break;
+        }
+        if (elect_one()) {
           if (is_x) {
             mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(C::kX1Bytes));
             tma_load_2d(s_x1 + st * C::kX1Bytes, &tmap_x1, &full[st], kt * kWqKTile, m0);
@@ -467,109 +476,181 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
                      &full[st]);
           }
         }
+        __syncwarp();
       }
-      // every copy this lane issued into the ring has landed before the CTA may exit
+    }
+    // every copy issued into the ring has landed before the CTA may exit
+    if (lane == 0) {
       const uint32_t first = g > static_cast<uint32_t>(ns) ? g - ns : 0;
       for (uint32_t i = first; i < g; ++i) {
-        if (static_cast<int>(i % kProducerLanes) != lane) continue;
         volatile int no_abort = 0;
         mbar_wait(&full[i % ns], (i / ns) & 1, &no_abort, p.err, kDevTimeoutDrain);
       }
     }
+    __syncwarp();
   } else if (warp == 1) {
     // ============================================================ MMA issuer
-    if (lane == 0) {
-      uint32_t g = 0, j = 0;
-      bool live = true;
-      while (live && walk.next(p, it)) {
-        const int ab = j % C::kNAcc;
-        if (!mbar_wait(&bar_accempty[ab], ((j / C::kNAcc) & 1) ^ 1, abort_flag, p.err, kDevTimeoutMma)) break;
+    // The whole warp walks the schedule and waits; the elected lane issues the
+    // MMAs and their commits (a commit tracks the MMAs of its own thread, and
+    // elect.sync of a converged warp always picks the same lane).
+    uint32_t g = 0, j = 0;
+    bool live = true;
+    while (live && walk.next(p, it)) {
+      const int ab = j % C::kNAcc;
+      if (!__all_sync(kFull,
+                      mbar_wait(&bar_accempty[ab], ((j / C::kNAcc) & 1) ^ 1, abort_flag, p.err, kDevTimeoutMma)))
+        break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem + ab * C::kAccCols;
+      for (int kt = it.kt0; kt < it.kt1;) {
+        const int nbs = min(C::kBatch, it.kt1 - kt);
+        // wait for every A stage of the batch, then issue it whole; afull of a
+        // step implies its x1 slab has landed (the dequantisers check)
+        bool ok = true;
+        for (int jj = 0; jj < nbs && ok; ++jj) {
+          const uint32_t gg = g + jj;
+          ok = mbar_wait(&bar_afull[gg % AS], (gg / AS) & 1, abort_flag, p.err, kDevTimeoutMma);
+        }
+        if (!__all_sync(kFull, ok)) {
+          live = false;
+          break;
+        }
         tc_fence_after();
-        const uint32_t d_tmem = tmem + ab * C::kAccCols;
-        for (int kt = it.kt0; kt < it.kt1 && live;) {
-          const int nbs = min(C::kBatch, it.kt1 - kt);
-          // wait for every x1 slab and A stage of the batch, then issue it whole
-          // afull of a step implies its x1 slab has landed (the dequantisers check)
-          for (int jj = 0; jj < nbs && live; ++jj) {
-            const uint32_t gg = g + jj;
-            live = mbar_wait(&bar_afull[gg % AS], (gg / AS) & 1, abort_flag, p.err, kDevTimeoutMma);
-          }
-          if (!live) break;
-          tc_fence_after();
-          for (int jj = 0; jj < nbs; ++jj) {
-            const uint32_t gg = g + jj;
-            const int sx = gg % SX;
-            const int as = gg % AS;
-            const uint32_t b_base = smem_u32(s_x1 + sx * C::kX1Bytes);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              mma_f16_ts(d_tmem, tmem + C::kACol0 + as * 32 + kk * 8, sdesc_kmajor_sw128(b_base + kk * 32), kIdesc,
-                         (kt + jj > it.kt0 || kk > 0) ? 1u : 0u);
-            }
+        for (int jj = 0; jj < nbs; ++jj) {
+          const uint32_t gg = g + jj;
+          const uint32_t b_base = smem_u32(s_x1 + (gg % SX) * C::kX1Bytes);
+          const uint32_t a_col = tmem + C::kACol0 + (gg % AS) * 32;
+          const uint32_t acc0 = (kt + jj > it.kt0) ? 1u : 0u;
+          if (elect_one()) {
+            mma_f16_ts(d_tmem, a_col, sdesc_kmajor_sw128(b_base), kIdesc, acc0);
+            mma_f16_ts(d_tmem, a_col + 8, sdesc_kmajor_sw128(b_base + 32), kIdesc, 1u);
+            mma_f16_ts(d_tmem, a_col + 16, sdesc_kmajor_sw128(b_base + 64), kIdesc, 1u);
+            mma_f16_ts(d_tmem, a_col + 24, sdesc_kmajor_sw128(b_base + 96), kIdesc, 1u);
             mma_commit(&bar_done[gg % RD]);
           }
-          kt += nbs;
-          g += nbs;
+          __syncwarp();
         }
-        if (!live) break;
-        mma_commit(&bar_accfull[ab]);
-        ++j;
+        kt += nbs;
+        g += nbs;
       }
+      if (!live) break;
+      if (elect_one()) mma_commit(&bar_accfull[ab]);
+      __syncwarp();
+      ++j;
+    }
+    if (elect_one()) {
       mma_commit(&bar_drain);
       volatile int no_abort = 0;
       mbar_wait(&bar_drain, 0, &no_abort, p.err, kDevTimeoutDrain);
     }
+    __syncwarp();
   } else if (warp < 6) {
     // ============================================================ epilogue
+    // Per chunk of kEpiRows accumulator columns (output rows): (1) each thread
+    // reads its weight column's values from TMEM, applies the per-column scale
+    // and writes them, fp32, into a staging tile [row][column]; (2) after a
+    // barrier of the four epilogue warps, each thread takes 8 consecutive
+    // columns of one row: + bias, + x3 (16-byte loads), one rounding, one
+    // 16-byte store.  Both global streams are coalesced whole rows.
     const int quad = warp & 3;
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+    const int et = threadIdx.x - 64;        // 0..127 over warps 2..5
+    const int col8 = (et & 15) * 8;          // phase 2: 8 columns ...
+    const int prow = et >> 4;                // ... of rows prow, prow + 8, ...
+    constexpr int kER = C::kEpiRows;
+    constexpr int kPasses = kER / 8;
+    float* stage = reinterpret_cast<float*>(s_stage);
     uint32_t j = 0;
     while (walk.next(p, it)) {
       const int ab = j % C::kNAcc;
-      bool ready =
-          mbar_wait_sleep(&bar_accfull[ab], (j / C::kNAcc) & 1, abort_flag, p.err, kDevTimeoutEpilogue, 256, 2048);
-      if (!__all_sync(kFull, ready && !*abort_flag)) break;
+      const bool ready =
+          mbar_wait_sleep(&bar_accfull[ab], (j / C::kNAcc) & 1, abort_flag, p.err, kDevTimeoutEpilogue, 64, 512);
+      // one decision for all four warps: they meet at named barriers below
+      if (!named_bar_and(1, 128, ready && !*abort_flag)) break;
       tc_fence_after();
       const int nb = it.tile % p.num_nb;
       const int64_t m0 = static_cast<int64_t>(it.tile / p.num_nb) * BN;
-      const int nl = quad * 32 + lane;  // column within the tile
+      const int nl = quad * 32 + lane;  // phase 1: weight column within the tile
       const int nn = nb * kWqNBlock + nl;
       const bool col_ok = nn < p.n;
-      float escale = 1.f, bias_v = 0.f;
+      const int nn8 = nb * kWqNBlock + col8;
+      const bool col8_ok = nn8 < p.n;  // n is a multiple of 32: all 8 columns or none
+      float escale = 1.f;
+      float bias8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) bias8[i] = 0.f;
       if (it.slot < 0) {
         if (p.mode != kPerGroup) {
           const ColConst cc = col_const<BF16, WK>(p, nn, col_ok);
           escale = (WK == kWFp8 || cc.fast) ? cc.s : 1.f;
         }
-        if (p.bias && col_ok) bias_v = act_f32(p.bias[nn], BF16);
+        if (p.bias && col8_ok) {
+          const uint4 b = *reinterpret_cast<const uint4*>(p.bias + nn8);
+          const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            bias8[2 * i] = act_f32(static_cast<uint16_t>(bw[i] & 0xFFFFu), BF16);
+            bias8[2 * i + 1] = act_f32(static_cast<uint16_t>(bw[i] >> 16), BF16);
+          }
+        }
       }
       float* part = (it.slot >= 0)
                         ? p.partial + (static_cast<int64_t>(it.tile) * p.max_slots + it.slot) * (BN * kWqNBlock)
                         : nullptr;
-      constexpr int kChunk = 16;  // accumulator columns (m rows) per tcgen05.ld
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += kChunk) {
-        uint32_t v[kChunk];
-        tmem_ld_x16(tmem + lane_addr + ab * C::kAccCols + c0, v);
+      for (int c0 = 0; c0 < BN; c0 += kER) {
+        const bool last = (c0 + kER >= BN);
+        // x3 of this thread's phase-2 rows, loaded first so its latency
+        // overlaps the TMEM read and the staging
+        uint4 xv[kPasses];
+#pragma unroll
+        for (int ps = 0; ps < kPasses; ++ps) {
+          const int64_t mm = m0 + c0 + ps * 8 + prow;
+          xv[ps] = (part == nullptr && p.x3 && col8_ok && mm < p.m)
+                       ? *reinterpret_cast<const uint4*>(p.x3 + mm * p.n + nn8)
+                       : make_uint4(0u, 0u, 0u, 0u);
+        }
+        uint32_t v[kER];
+        if constexpr (kER == 32)
+          tmem_ld_x32(tmem + lane_addr + ab * C::kAccCols + c0, v);
+        else
+          tmem_ld_x16(tmem + lane_addr + ab * C::kAccCols + c0, v);
         tmem_wait_ld();
+        if (last) {
+          // the whole accumulator is in registers or staged: hand it back
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar_accempty[ab]);
+        }
         if (part) {
 #pragma unroll
-          for (int q = 0; q < kChunk; ++q) part[(c0 + q) * kWqNBlock + nl] = __uint_as_float(v[q]);
-        } else if (col_ok) {
+          for (int q = 0; q < kER; ++q) part[(c0 + q) * kWqNBlock + nl] = __uint_as_float(v[q]);
+          continue;
+        }
 #pragma unroll
-          for (int q = 0; q < kChunk; ++q) {
-            const int64_t mm = m0 + c0 + q;
-            if (mm < p.m) {
-              float y = __uint_as_float(v[q]) * escale + bias_v;
-              if (p.x3) y += act_f32(p.x3[mm * p.n + nn], BF16);
-              p.out[mm * p.n + nn] = f32_act(y, BF16);
+        for (int q = 0; q < kER; ++q) stage[q * kWqNBlock + nl] = __uint_as_float(v[q]) * escale;
+        named_bar_sync(1, 128);
+#pragma unroll
+        for (int ps = 0; ps < kPasses; ++ps) {
+          const int row = ps * 8 + prow;
+          const int64_t mm = m0 + c0 + row;
+          if (col8_ok && mm < p.m) {
+            const float4 lo = *reinterpret_cast<const float4*>(stage + row * kWqNBlock + col8);
+            const float4 hi = *reinterpret_cast<const float4*>(stage + row * kWqNBlock + col8 + 4);
+            const float y[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+            const uint32_t xw[4] = {xv[ps].x, xv[ps].y, xv[ps].z, xv[ps].w};
+            uint32_t o[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float a = y[2 * i] + bias8[2 * i] + act_f32(static_cast<uint16_t>(xw[i] & 0xFFFFu), BF16);
+              const float b = y[2 * i + 1] + bias8[2 * i + 1] + act_f32(static_cast<uint16_t>(xw[i] >> 16), BF16);
+              o[i] = pack2<BF16>(a, b);
             }
+            *reinterpret_cast<uint4*>(p.out + mm * p.n + nn8) = make_uint4(o[0], o[1], o[2], o[3]);
           }
         }
+        named_bar_sync(1, 128);  // the staging tile is rewritten by the next chunk
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_accempty[ab]);
       ++j;
     }
   } else {
@@ -619,15 +700,7 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
         for (int c = 0; c < kChunks; ++c) ch[c] = *reinterpret_cast<const uint4*>(wt + (c * kWqNBlock + r) * 16);
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar_wempty[sw]);
-        // 2) dequantise into an A stage of TMEM
-        got = mbar_wait_sleep(&bar_xfull[g % SX], (g / SX) & 1, abort_flag, p.err, kDevTimeoutDequant, 32, 256);
-        if (got && g >= static_cast<uint32_t>(AS))
-          got = mbar_wait_sleep(&bar_done[(g - AS) % RD], ((g - AS) / RD) & 1, abort_flag, p.err,
-                                kDevTimeoutDequant, 32, 256);
-        if (!__all_sync(kFull, got)) {  // tcgen05.st below is warp-collective
-          live = false;
-          break;
-        }
+        // 2) dequantise in registers: needs nothing but the weights
         uint32_t a[32];
         if constexpr (WK == kW4) {
           if (grp) {
@@ -655,10 +728,22 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 4; ++c) dq_fp8<BF16>(ch[c], a + 8 * c);
         }
+        // 3) the A stage is free once the MMA of step g - AS is done
+        got = g < static_cast<uint32_t>(AS) ||
+              mbar_wait(&bar_done[(g - AS) % RD], ((g - AS) / RD) & 1, abort_flag, p.err, kDevTimeoutDequant);
+        if (!__all_sync(kFull, got)) {  // tcgen05.st below is warp-collective
+          live = false;
+          break;
+        }
         tmem_st_x32(tmem + lane_addr + C::kACol0 + as * 32, a);
         tmem_wait_st();
         tc_fence_before();
-        __syncwarp();
+        // 4) the stage may be issued once this step's x1 slab has landed too
+        got = mbar_wait(&bar_xfull[g % SX], (g / SX) & 1, abort_flag, p.err, kDevTimeoutDequant);
+        if (!__all_sync(kFull, got)) {
+          live = false;
+          break;
+        }
         if (lane == 0) mbar_arrive(&bar_afull[as]);
       }
     }
