@@ -81,16 +81,23 @@ struct Cfg {
   static constexpr int kEpiRows = 16;
   static constexpr int kStageBytes = kEpiRows * 128 * 4;
   static constexpr int kSmemBudget = 224 * 1024 - kStageBytes;
-  static constexpr int kWStages =
-      BN <= 64 ? cmin(32, (kSmemBudget - 8 * kX1Bytes) / kTile) : ((WK == kW4) ? 10 : 6);
-  static constexpr int kXStages = cmin(16, (kSmemBudget - kWStages * kTile) / kX1Bytes);
+  // A weight stage holds kWQ consecutive k steps (16 KB) and is filled by one
+  // or two bulk copies: a copy instruction holds its issuing thread for hundreds
+  // of cycles whatever its size, so fewer, larger copies stream faster.
+  static constexpr int kWQ = 16384 / kTile;
+  static constexpr int kWStageBytes = kWQ * kTile;
+  static constexpr int kWStages = BN <= 64 ? cmin(12, (kSmemBudget - 8 * kX1Bytes) / kWStageBytes) : 3;
+  static constexpr int kXStages = cmin(16, (kSmemBudget - kWStages * kWStageBytes) / kX1Bytes);
   // The MMA issuer waits once per batch of k steps (half the A stages) and then
   // issues the whole batch: every barrier wait in the issuing thread costs the
   // tensor pipe its queued overlap, so a wait has to be followed by roughly
   // 800+ cycles of MMA work to keep the pipe busy.
   static constexpr int kBatch = cmax(1, cmin(kAStages / 2, kXStages / 2));
-  static constexpr int kThreads = 32 * (7 + 4 * DG);
-  static constexpr int kSmemBytes = kXStages * kX1Bytes + kWStages * kTile + kStageBytes + 1024;
+  // warps: 0 and kXWarp2 x1 producers, 1 MMA, 2..5 epilogue, 6 weight producer,
+  // 7 .. 7 + 4 DG - 1 dequantisation
+  static constexpr int kXWarp2 = 7 + 4 * DG;
+  static constexpr int kThreads = 32 * (8 + 4 * DG);
+  static constexpr int kSmemBytes = kXStages * kX1Bytes + kWStages * kWStageBytes + kStageBytes + 1024;
   static_assert(kAStages >= DG && kAStages % DG == 0, "A stages");
   static_assert(kACol0 + kAStages * 32 <= 512, "TMEM budget");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -388,7 +395,7 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* s_x1 = smem;                  // SX x (BN x 128 B), 1024-aligned slabs
   uint8_t* s_w = s_x1 + SX * C::kX1Bytes;  // SW x packed weight tile
-  uint8_t* s_stage = s_w + SW * kTile;     // epilogue staging tile (fp32)
+  uint8_t* s_stage = s_w + SW * C::kWStageBytes;  // epilogue staging tile (fp32)
 
   __shared__ __align__(8) uint64_t bar_xfull[SX];
   __shared__ __align__(8) uint64_t bar_done[RD];  // one commit per k step: x1 slab and A stage free
@@ -410,7 +417,7 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
     }
     for (int i = 0; i < SW; ++i) {
       mbar_init(&bar_wfull[i], 1);
-      mbar_init(&bar_wempty[i], 4);
+      mbar_init(&bar_wempty[i], 4 * C::kWQ);
     }
     for (int i = 0; i < AS; ++i) {
       mbar_init(&bar_afull[i], 4);
@@ -438,53 +445,93 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
   walk.init(p);
   Item it;
 
-  if (warp == 0 || warp == 6) {
-    // ============================================================ producers
-    // warp 0: x1 tiles (one 2-D tensor copy per k step) for the MMA;
-    // warp 6: packed weight tiles (one 1-D bulk copy per k step) for the dequantisers.
-    // The whole warp walks the ring and waits; one elected lane issues each
-    // copy, so its operands are warp-uniform.
-    const bool is_x = (warp == 0);
-    if (is_x && elect_one()) prefetch_tensormap(&tmap_x1);
+  if (warp == 0 || warp == C::kXWarp2) {
+    // ============================================================ x1 producers
+    // Two warps take alternate k steps: one 2-D tensor copy (BN rows x 64 k,
+    // 128-byte swizzle) per step into the x1 ring.  The whole warp walks the
+    // ring and waits; one elected lane issues, so its operands are warp-uniform.
+    const uint32_t xp = (warp == 0) ? 0u : 1u;
+    if (xp == 0 && elect_one()) prefetch_tensormap(&tmap_x1);
     __syncwarp();
-    const int ns = is_x ? SX : SW;
-    uint64_t* full = is_x ? bar_xfull : bar_wfull;
     uint32_t g = 0;
     bool live = true;
     while (live && walk.next(p, it)) {
-      const int nb = it.tile % p.num_nb;
       const int32_t m0 = static_cast<int32_t>(static_cast<int64_t>(it.tile / p.num_nb) * BN);
       for (int kt = it.kt0; kt < it.kt1; ++kt, ++g) {
-        const int st = g % ns;
-        // x1 slab free once the MMA of step g - SX is done; weight stage once read
-        const bool ok = is_x ? (g < static_cast<uint32_t>(SX) ||
-                                mbar_wait(&bar_done[(g - SX) % RD], ((g - SX) / RD) & 1, abort_flag, p.err,
-                                          kDevTimeoutProducer))
-                             : mbar_wait_sleep(&bar_wempty[st], ((g / ns) & 1) ^ 1, abort_flag, p.err,
-                                               kDevTimeoutProducer, 32, 256);
+        if ((g & 1u) != xp) continue;
+        const int st = g % SX;
+        // the slab is free once the MMA of step g - SX is done
+        const bool ok = g < static_cast<uint32_t>(SX) ||
+                        mbar_wait(&bar_done[(g - SX) % RD], ((g - SX) / RD) & 1, abort_flag, p.err,
+                                  kDevTimeoutProducer);
         if (!__all_sync(kFull, ok)) {
           live = false;
           break;
         }
         if (elect_one()) {
-          if (is_x) {
-            mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(C::kX1Bytes));
-            tma_load_2d(s_x1 + st * C::kX1Bytes, &tmap_x1, &full[st], kt * kWqKTile, m0);
-          } else {
-            mbar_arrive_expect_tx(&full[st], static_cast<uint32_t>(kTile));
-            bulk_g2s(s_w + st * kTile, p.wpack + (static_cast<int64_t>(nb) * p.kt_total + kt) * kTile, kTile,
-                     &full[st]);
-          }
+          mbar_arrive_expect_tx(&bar_xfull[st], static_cast<uint32_t>(C::kX1Bytes));
+          tma_load_2d(s_x1 + st * C::kX1Bytes, &tmap_x1, &bar_xfull[st], kt * kWqKTile, m0);
         }
         __syncwarp();
       }
     }
-    // every copy issued into the ring has landed before the CTA may exit
+    // every copy this warp issued has landed before the CTA may exit
     if (lane == 0) {
-      const uint32_t first = g > static_cast<uint32_t>(ns) ? g - ns : 0;
+      const uint32_t first = g > static_cast<uint32_t>(SX) ? g - SX : 0;
       for (uint32_t i = first; i < g; ++i) {
+        if ((i & 1u) != xp) continue;
         volatile int no_abort = 0;
-        mbar_wait(&full[i % ns], (i / ns) & 1, &no_abort, p.err, kDevTimeoutDrain);
+        mbar_wait(&bar_xfull[i % SX], (i / SX) & 1, &no_abort, p.err, kDevTimeoutDrain);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 6) {
+    // ============================================================ weight producer
+    // Stage s holds this CTA's k steps s*kWQ .. s*kWQ + kWQ - 1: one bulk copy per
+    // run of consecutive k steps of one tile (packed tiles of one column block
+    // are contiguous along k), so usually one copy per stage.
+    constexpr int Q = C::kWQ;
+    uint32_t s = 0;
+    bool have = walk.next(p, it);
+    int kt = have ? it.kt0 : 0;
+    while (have) {
+      const int st = s % SW;
+      const bool ok = mbar_wait_sleep(&bar_wempty[st], ((s / SW) & 1) ^ 1, abort_flag, p.err, kDevTimeoutProducer,
+                                      32, 256);
+      if (!__all_sync(kFull, ok)) break;
+      const uint8_t* src[Q];
+      int cnt[Q];
+      int np = 0, n_in = 0;
+      while (n_in < Q && have) {
+        const int nb = it.tile % p.num_nb;
+        const int run = min(Q - n_in, it.kt1 - kt);
+        src[np] = p.wpack + (static_cast<int64_t>(nb) * p.kt_total + kt) * kTile;
+        cnt[np] = run;
+        ++np;
+        n_in += run;
+        kt += run;
+        if (kt >= it.kt1) {
+          have = walk.next(p, it);
+          if (have) kt = it.kt0;
+        }
+      }
+      if (elect_one()) {
+        mbar_arrive_expect_tx(&bar_wfull[st], static_cast<uint32_t>(n_in * kTile));
+        int off = 0;
+        for (int i = 0; i < np; ++i) {
+          bulk_g2s(s_w + st * C::kWStageBytes + off * kTile, src[i], static_cast<uint32_t>(cnt[i] * kTile),
+                   &bar_wfull[st]);
+          off += cnt[i];
+        }
+      }
+      __syncwarp();
+      ++s;
+    }
+    if (lane == 0) {
+      const uint32_t first = s > static_cast<uint32_t>(SW) ? s - SW : 0;
+      for (uint32_t i = first; i < s; ++i) {
+        volatile int no_abort = 0;
+        mbar_wait(&bar_wfull[i % SW], (i / SW) & 1, &no_abort, p.err, kDevTimeoutDrain);
       }
     }
     __syncwarp();
@@ -685,15 +732,16 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
           grow.advance(2 * DG, gq);
           so_next = load_group_so(p, kt + DG, grow, gq, nn, col_ok);
         }
-        const int sw = g % SW;
+        const int sw = (g / C::kWQ) % SW;
         const int as = g % AS;
         // 1) weight tile -> registers, then hand the stage back to the producer
-        bool got = mbar_wait_sleep(&bar_wfull[sw], (g / SW) & 1, abort_flag, p.err, kDevTimeoutDequant, 32, 256);
+        bool got = mbar_wait_sleep(&bar_wfull[sw], (g / C::kWQ / SW) & 1, abort_flag, p.err, kDevTimeoutDequant,
+                                   32, 256);
         if (!__all_sync(kFull, got)) {
           live = false;
           break;
         }
-        const uint8_t* wt = s_w + sw * kTile;
+        const uint8_t* wt = s_w + sw * C::kWStageBytes + (g % C::kWQ) * kTile;
         constexpr int kChunks = (WK == kW4) ? 2 : 4;
         uint4 ch[kChunks];
 #pragma unroll
