@@ -117,6 +117,54 @@ def test_wqmm_small_parity(spec):
     check_wqmm(case)
 
 
+# ---------------------------------------------------------------- CTA pairs
+# m > 128 selects the 192-row m tile; with whole tiles per CTA (stream-K off)
+# and WQMM_PAIR=1, two CTAs of a cluster share each MMA (cta_group::2), each
+# holding half of the x1 slab and its own 128 weight columns.  Odd column-block counts leave
+# the second CTA of the last pair without weights (its outputs are masked).
+PAIRS = [
+    # name, x1_shape, n, act, wdt, mode, G, extras
+    ("pair_i4_group128_bf16_ragged", (400, 640), 384, "bf16", "i4", "group", 128,
+     {"scale_range": (0.005, 0.05), "offset_range": (-4, 4)}),
+    ("pair_i8_tensor_bf16_x3", (300, 320), 256, "bf16", "i8", "tensor", 0, {"scale_const": 0.01, "offset_const": 3.0}),
+    ("pair_i8_chan_f16_oddblocks", (193, 256), 640, "f16", "i8", "channel", 0, {}),
+    ("pair_i4_group64_f16_fractional", (250, 256), 256, "f16", "i4", "group", 64, {"fractional_offset": True}),
+    ("pair_fp8_chan_bf16", (385, 128), 384, "bf16", "fp8", "channel", 0, {"offset": False}),
+    ("pair_i8_group32_bf16_3d", (3, 70, 192), 512, "bf16", "i8", "group", 32, {}),
+]
+
+
+@pytest.fixture
+def whole_tiles(monkeypatch):
+    monkeypatch.setenv("WQMM_STREAMK", "0")
+    monkeypatch.setenv("WQMM_PAIR", "1")
+    yield
+
+
+@pytest.mark.parametrize("spec", PAIRS, ids=[s[0] for s in PAIRS])
+def test_wqmm_cta_pair_parity(spec, whole_tiles):
+    name, x1s, n, act, wdt, mode, G, extra = spec
+    case = WL.make_wqmm_case(name=name, x1_shape=x1s, n=n, act=act, wdt=wdt, mode=mode, group_size=G,
+                             seed=zlib.crc32(name.encode()) % 10000, **extra)
+    check_wqmm(case)
+
+
+def test_wqmm_cta_pair_matches_single_cta(monkeypatch):
+    # the same problem with and without CTA pairs: both within tolerance of the
+    # oracle, and close to each other
+    monkeypatch.setenv("WQMM_STREAMK", "0")
+    monkeypatch.setenv("WQMM_PAIR", "1")
+    case = WL.make_wqmm_case(name="pair_vs_single", x1_shape=(512, 1024), n=512, act="bf16", wdt="i4", mode="group",
+                             group_size=128, scale_range=(0.005, 0.05), offset_range=(-4, 4), seed=11)
+    a = dec(run_wqmm(case), case.act)
+    monkeypatch.setenv("WQMM_PAIR", "0")
+    b = dec(run_wqmm(case), case.act)
+    ye, _ = oracle.wqmm(case)
+    assert rel_err(a, ye) <= TOL[case.act]
+    assert rel_err(b, ye) <= TOL[case.act]
+    assert rel_err(a, b) <= TOL[case.act]
+
+
 @pytest.mark.parametrize("wdt,mode,G", [("i8", "group", 32), ("i4", "group", 64), ("fp8", "channel", 0),
                                         ("i8", "channel", 0)])
 def test_wqmm_transposed_weight(wdt, mode, G):

@@ -8,7 +8,9 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <tuple>
 #include <new>
 #include <string>
 #include <thread>
@@ -79,6 +81,8 @@ struct wqmm_executor {
   int bn = 256;
   int grid = 1;        // persistent CTAs of the GEMM
   int stream_k = 0;    // 1: k steps of all tiles split evenly over the grid, partials + fix-up
+  int pair = 0;        // 1: clusters of two CTAs share each MMA (256 weight columns per pair tile)
+  int num_pnb = 0;     // pair: 256-column blocks
   int num_tiles = 0;
   int max_slots = 0;
   // qmm
@@ -170,6 +174,25 @@ int sm_count() {
 }
 
 uint64_t round_up(uint64_t v, uint64_t a) { return (v + a - 1) / a * a; }
+
+// Resident CTA pairs of the pair-mode GEMM, per (device, m tile, weight kind,
+// activation type); 0 when there is no pair mode or no device.
+int pair_slots(int bn, int wk, bool bf16) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int, int>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  const auto key = std::make_tuple(dev, bn, wk, bf16 ? 1 : 0);
+  std::lock_guard<std::mutex> lock(mu);
+  auto f = cache.find(key);
+  if (f != cache.end()) return f->second;
+  const int v = wqmm_pair_slots(bn, wk, bf16);
+  cache[key] = v;
+  return v;
+}
 
 uint64_t packed_bytes_for(int x2_dtype, int64_t k, int64_t n, bool for_qmm) {
   if (for_qmm) {
@@ -419,6 +442,24 @@ extern "C" wqmm_status wqmm_get_workspace_size(const wqmm_tensor* x1, const wqmm
         if (c > ms) ms = static_cast<int>(c);
       }
       ex->max_slots = ms;
+    }
+    // 192-row m tiles over whole tiles can run as clusters of two CTAs that
+    // share each MMA (each CTA holds half of the x1 slab).  Measured on B200 it
+    // is not faster than single CTAs (both are bound by instruction issue in the
+    // dequantisation), so it is opt-in: WQMM_PAIR=1.
+    const char* pair_env = std::getenv("WQMM_PAIR");
+    const bool want_pair = pair_env && std::atoi(pair_env) == 1;
+    if (!ex->stream_k && want_pair && ex->bn == 192 && num_nb >= 2) {
+      const int wk = x2->dtype == WQMM_DT_I4 ? kW4 : (x2->dtype == WQMM_DT_I8 ? kW8 : kWFp8);
+      const int ps = pair_slots(ex->bn, wk, adt == WQMM_DT_BF16);
+      if (ps > 0) {
+        const int64_t pnb = (num_nb + 1) / 2;
+        const int64_t ptiles = num_mb * pnb;
+        ex->pair = 1;
+        ex->num_pnb = static_cast<int>(pnb);
+        ex->num_tiles = static_cast<int>(ptiles);
+        ex->grid = static_cast<int>(2 * (ptiles < ps ? ptiles : ps));
+      }
     }
     if (!ex->x2_packed) {
       ex->ws_pack = {ws, packed_bytes_for(x2->dtype, k, n, false)};
@@ -672,7 +713,7 @@ wqmm_status run_wqmm(void* ws, wqmm_executor* ex, cudaStream_t s) {
   }
   CUtensorMap tmap;
   wqmm_status st = make_tmap(&tmap, ex->x1, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                             2, ex->m, ex->k, kWqKTile, ex->bn);
+                             2, ex->m, ex->k, kWqKTile, ex->pair ? ex->bn / 2 : ex->bn);
   if (st) return st;
   WqParams p{};
   p.wpack = wpack;
@@ -690,6 +731,8 @@ wqmm_status run_wqmm(void* ws, wqmm_executor* ex, cudaStream_t s) {
   p.num_nb = (ex->n + kWqNBlock - 1) / kWqNBlock;
   p.num_mb = static_cast<int>((ex->m + ex->bn - 1) / ex->bn);
   p.num_tiles = ex->num_tiles;
+  p.pair = ex->pair;
+  p.num_pnb = ex->num_pnb;
   p.stream_k = ex->stream_k;
   p.max_slots = ex->max_slots;
   p.mode = ex->mode;

@@ -40,6 +40,10 @@ struct WqParams {
   int num_nb;             // ceil(n / 128)
   int num_mb;             // ceil(m / BN)
   int num_tiles;          // num_mb * num_nb; tile t = (mb = t / num_nb, nb = t % num_nb)
+                          // pair: num_mb * num_pnb pair tiles (mb = t / num_pnb,
+                          // column blocks 2 * (t % num_pnb) + cluster rank)
+  int pair;               // 1: clusters of two CTAs share each MMA (cta_group::2)
+  int num_pnb;            // pair: ceil(num_nb / 2)
   int stream_k;           // 0: whole tiles round-robin over the grid; 1: k-steps split evenly
   int max_slots;          // stream-K: partial slots per tile
   int mode;               // QuantMode
@@ -121,6 +125,9 @@ cudaError_t launch_transpose_u16(const uint16_t* src, uint16_t* dst, int rows, i
 // Launch configuration of the anti-quant GEMM for a BN-row m tile: CTAs per SM
 // the kernel's shared/tensor memory allows (the grid is a multiple of it).
 int wqmm_ctas_per_sm(int bn, int wk);
+// Clusters of two CTAs of the pair-mode anti-quant GEMM that fit at once (0 if
+// the m tile has no pair mode or clusters cannot be scheduled).
+int wqmm_pair_slots(int bn, int wk, bool act_bf16);
 cudaError_t launch_wqmm_gemm(const CUtensorMap& tmap_x1, const WqParams& p, int bn, int wk, bool act_bf16,
                              int grid, cudaStream_t s);
 cudaError_t launch_wqmm_fixup(const FixupParams& p, cudaStream_t s);

@@ -59,10 +59,12 @@ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 
 constexpr int cmax(int a, int b) { return a > b ? a : b; }
 
-template <int BN, int DG, int WK>
+template <int BN, int DG, int WK, bool PAIR = false>
 struct Cfg {
   static constexpr int kTile = wq_tile_bytes(WK);
-  static constexpr int kX1Bytes = BN * 128;
+  // x1 slab of one k step held by this CTA: BN rows, or BN / 2 when a CTA pair
+  // shares the MMA (each CTA holds half of the B operand)
+  static constexpr int kX1Bytes = (PAIR ? BN / 2 : BN) * 128;
   static constexpr int kAccCols = BN < 32 ? 32 : BN;
   static constexpr int kNAcc = (2 * kAccCols + 4 * 32 <= 512) ? 2 : 1;
   static constexpr int kACol0 = kNAcc * kAccCols;
@@ -324,15 +326,18 @@ struct Item {
 
 // Identical walk of this CTA's work in every role.
 struct Walker {
-  int64_t cur, end, T;
-  __device__ __forceinline__ void init(const WqParams& p) {
+  int64_t cur, end, T, step;
+  // pair: both CTAs of a pair walk the same pair tiles (no stream-K then)
+  __device__ __forceinline__ void init(const WqParams& p, bool pair) {
     if (p.stream_k) {
       T = static_cast<int64_t>(p.num_tiles) * p.kt_total;
       cur = sk_start(blockIdx.x, T, gridDim.x);
       end = sk_start(blockIdx.x + 1, T, gridDim.x);
+      step = gridDim.x;
     } else {
       T = 0;
-      cur = blockIdx.x;
+      cur = pair ? (blockIdx.x >> 1) : blockIdx.x;
+      step = pair ? (gridDim.x >> 1) : gridDim.x;
       end = p.num_tiles;
     }
   }
@@ -343,7 +348,7 @@ struct Walker {
       it.kt0 = 0;
       it.kt1 = p.kt_total;
       it.slot = -1;
-      cur += gridDim.x;
+      cur += step;
       return true;
     }
     const int64_t tile = cur / p.kt_total;
@@ -377,10 +382,10 @@ __device__ __forceinline__ ColConst col_const(const WqParams& p, int nn, bool co
   return c;
 }
 
-template <int BN, int DG, int WK, bool BF16>
-__global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
+template <int BN, int DG, int WK, bool BF16, bool PAIR>
+__global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR>::kThreads, 1)
     wqmm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x1, const WqParams p) {
-  using C = Cfg<BN, DG, WK>;
+  using C = Cfg<BN, DG, WK, PAIR>;
   constexpr int SX = C::kXStages;
   constexpr int SW = C::kWStages;
   constexpr int AS = C::kAStages;
@@ -389,7 +394,7 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
   // that barrier lapped, since step g - X + RD needs data it has not yet made.
   constexpr int RD = SX + AS;
   constexpr int kTile = C::kTile;
-  constexpr uint32_t kIdesc = idesc_make(1u, BF16 ? 1u : 0u, 128u, static_cast<uint32_t>(BN));
+  constexpr uint32_t kIdesc = idesc_make(1u, BF16 ? 1u : 0u, PAIR ? 256u : 128u, static_cast<uint32_t>(BN));
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -410,6 +415,11 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // CTA pairs: rank 0 issues the pair's MMAs; the A-stage and accumulator-free
+  // barriers of rank 0 count the arrivals of both CTAs
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool mma_cta = (rank == 0);
+  constexpr uint32_t kArrivers = PAIR ? 8u : 4u;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < SX; ++i) {
@@ -420,30 +430,50 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
       mbar_init(&bar_wempty[i], 4 * C::kWQ);
     }
     for (int i = 0; i < AS; ++i) {
-      mbar_init(&bar_afull[i], 4);
+      mbar_init(&bar_afull[i], kArrivers);
     }
     for (int i = 0; i < RD; ++i) mbar_init(&bar_done[i], 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_accfull[i], 1);
-      mbar_init(&bar_accempty[i], 4);
+      mbar_init(&bar_accempty[i], kArrivers);
     }
     mbar_init(&bar_drain, 1);
     abort_sh = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(&tmem_base_sh, C::kTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc2(&tmem_base_sh, C::kTmemCols);
+      tmem_relinquish2();
+    } else {
+      tmem_alloc(&tmem_base_sh, C::kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // the other CTA's barriers are initialised
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
   volatile int* abort_flag = &abort_sh;
 
   Walker walk;
-  walk.init(p);
+  walk.init(p, PAIR);
   Item it;
+  // tile -> (m block, 128-column weight block of this CTA)
+  auto tile_mb = [&](int t) { return PAIR ? t / p.num_pnb : t / p.num_nb; };
+  auto tile_nb = [&](int t) { return PAIR ? 2 * (t % p.num_pnb) + static_cast<int>(rank) : t % p.num_nb; };
+  // arrival on a barrier that counts the arrivals of both CTAs of a pair, for
+  // tensor-memory hand-offs (A stage written, accumulator read): the data is
+  // ordered by tcgen05.wait::st/ld and tcgen05.fence::before_thread_sync, so
+  // the arrival is relaxed -- a release would first wait for the arriving
+  // warp's outstanding prefetch loads (hundreds of cycles from L2)
+  auto arrive_mma_cta = [&](uint64_t* bar) {
+    if constexpr (PAIR)
+      mbar_arrive_remote_relaxed(mapa_shared(smem_u32(bar), 0u));
+    else
+      mbar_arrive_relaxed(bar);
+  };
 
   if (warp == 0 || warp == C::kXWarp2) {
     // ============================================================ x1 producers
@@ -456,7 +486,8 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
     uint32_t g = 0;
     bool live = true;
     while (live && walk.next(p, it)) {
-      const int32_t m0 = static_cast<int32_t>(static_cast<int64_t>(it.tile / p.num_nb) * BN);
+      const int32_t m0 = static_cast<int32_t>(static_cast<int64_t>(tile_mb(it.tile)) * BN +
+                                              (PAIR ? static_cast<int64_t>(rank) * (BN / 2) : 0));
       for (int kt = it.kt0; kt < it.kt1; ++kt, ++g) {
         if ((g & 1u) != xp) continue;
         const int st = g % SX;
@@ -503,9 +534,11 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
       int cnt[Q];
       int np = 0, n_in = 0;
       while (n_in < Q && have) {
-        const int nb = it.tile % p.num_nb;
+        const int nb = tile_nb(it.tile);
         const int run = min(Q - n_in, it.kt1 - kt);
-        src[np] = p.wpack + (static_cast<int64_t>(nb) * p.kt_total + kt) * kTile;
+        // a column block past n (pairs over an odd block count) loads nothing:
+        // its stage keeps stale bytes and its outputs are never written
+        src[np] = nb < p.num_nb ? p.wpack + (static_cast<int64_t>(nb) * p.kt_total + kt) * kTile : nullptr;
         cnt[np] = run;
         ++np;
         n_in += run;
@@ -516,11 +549,14 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
         }
       }
       if (elect_one()) {
-        mbar_arrive_expect_tx(&bar_wfull[st], static_cast<uint32_t>(n_in * kTile));
+        int bytes = 0;
+        for (int i = 0; i < np; ++i) bytes += src[i] ? cnt[i] * kTile : 0;
+        mbar_arrive_expect_tx(&bar_wfull[st], static_cast<uint32_t>(bytes));
         int off = 0;
         for (int i = 0; i < np; ++i) {
-          bulk_g2s(s_w + st * C::kWStageBytes + off * kTile, src[i], static_cast<uint32_t>(cnt[i] * kTile),
-                   &bar_wfull[st]);
+          if (src[i])
+            bulk_g2s(s_w + st * C::kWStageBytes + off * kTile, src[i], static_cast<uint32_t>(cnt[i] * kTile),
+                     &bar_wfull[st]);
           off += cnt[i];
         }
       }
@@ -539,58 +575,100 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
     // ============================================================ MMA issuer
     // The whole warp walks the schedule and waits; the elected lane issues the
     // MMAs and their commits (a commit tracks the MMAs of its own thread, and
-    // elect.sync of a converged warp always picks the same lane).
-    uint32_t g = 0, j = 0;
-    bool live = true;
-    while (live && walk.next(p, it)) {
-      const int ab = j % C::kNAcc;
-      if (!__all_sync(kFull,
-                      mbar_wait(&bar_accempty[ab], ((j / C::kNAcc) & 1) ^ 1, abort_flag, p.err, kDevTimeoutMma)))
-        break;
-      tc_fence_after();
-      const uint32_t d_tmem = tmem + ab * C::kAccCols;
-      for (int kt = it.kt0; kt < it.kt1;) {
-        const int nbs = min(C::kBatch, it.kt1 - kt);
-        // wait for every A stage of the batch, then issue it whole; afull of a
-        // step implies its x1 slab has landed (the dequantisers check)
-        bool ok = true;
-        for (int jj = 0; jj < nbs && ok; ++jj) {
-          const uint32_t gg = g + jj;
-          ok = mbar_wait(&bar_afull[gg % AS], (gg / AS) & 1, abort_flag, p.err, kDevTimeoutMma);
-        }
-        if (!__all_sync(kFull, ok)) {
-          live = false;
-          break;
-        }
+    // elect.sync of a converged warp always picks the same lane).  With CTA
+    // pairs only rank 0 issues: one MMA covers both CTAs, and each commit
+    // arrives on the barrier of both.
+    if (mma_cta) {
+      // barrier waits for arrivals that may come from the other CTA of the pair
+      auto wait_pair = [&](uint64_t* bar, uint32_t parity) {
+        return mbar_wait(bar, parity, abort_flag, p.err, kDevTimeoutMma);
+      };
+      auto mma = [&](uint32_t d, uint32_t a, uint64_t b, uint32_t acc) {
+        if constexpr (PAIR)
+          mma_f16_ts2(d, a, b, kIdesc, acc);
+        else
+          mma_f16_ts(d, a, b, kIdesc, acc);
+      };
+      auto commit = [&](uint64_t* bar) {
+        if constexpr (PAIR)
+          mma_commit2_mc(bar, static_cast<uint16_t>(0x3));
+        else
+          mma_commit(bar);
+      };
+      // The issuing warp shares its sub-partition with busy dequantisation
+      // warps, so its loop is kept short: ring positions advance by one
+      // instead of by modulo, and each MMA's operands are one add away from
+      // precomputed bases (a descriptor's start address counts 16-byte units).
+      const uint64_t bdesc0 = sdesc_kmajor_sw128(smem_u32(s_x1));
+      constexpr uint64_t kSlabDesc = C::kX1Bytes >> 4;
+      const uint32_t a_base = tmem + C::kACol0;
+      uint32_t xs = 0, as_ = 0, rd = 0, a_par = 0;  // ring positions of the next step
+      uint32_t j = 0;
+      bool live = true;
+      while (live && walk.next(p, it)) {
+        const int ab = j % C::kNAcc;
+        if (!__all_sync(kFull, wait_pair(&bar_accempty[ab], ((j / C::kNAcc) & 1) ^ 1))) break;
         tc_fence_after();
-        for (int jj = 0; jj < nbs; ++jj) {
-          const uint32_t gg = g + jj;
-          const uint32_t b_base = smem_u32(s_x1 + (gg % SX) * C::kX1Bytes);
-          const uint32_t a_col = tmem + C::kACol0 + (gg % AS) * 32;
-          const uint32_t acc0 = (kt + jj > it.kt0) ? 1u : 0u;
-          if (elect_one()) {
-            mma_f16_ts(d_tmem, a_col, sdesc_kmajor_sw128(b_base), kIdesc, acc0);
-            mma_f16_ts(d_tmem, a_col + 8, sdesc_kmajor_sw128(b_base + 32), kIdesc, 1u);
-            mma_f16_ts(d_tmem, a_col + 16, sdesc_kmajor_sw128(b_base + 64), kIdesc, 1u);
-            mma_f16_ts(d_tmem, a_col + 24, sdesc_kmajor_sw128(b_base + 96), kIdesc, 1u);
-            mma_commit(&bar_done[gg % RD]);
+        const uint32_t d_tmem = tmem + ab * C::kAccCols;
+        for (int kt = it.kt0; kt < it.kt1;) {
+          const int nbs = min(C::kBatch, it.kt1 - kt);
+          // wait for every A stage of the batch, then issue it whole; afull of a
+          // step implies its x1 slab has landed (the dequantisers check)
+          bool ok = true;
+          {
+            uint32_t s = as_, par = a_par;
+            for (int jj = 0; jj < nbs && ok; ++jj) {
+              ok = wait_pair(&bar_afull[s], par);
+              if (++s == AS) {
+                s = 0;
+                par ^= 1u;
+              }
+            }
           }
-          __syncwarp();
+          if (!__all_sync(kFull, ok)) {
+            live = false;
+            break;
+          }
+          tc_fence_after();
+          // operands are computed by the whole warp (warp-uniform); only the
+          // tcgen05 instructions sit in the elected lane's branch
+          for (int jj = 0; jj < nbs; ++jj) {
+            const uint64_t bd = bdesc0 + xs * kSlabDesc;
+            const uint32_t a = a_base + as_ * 32;
+            const uint32_t acc0 = (kt + jj > it.kt0) ? 1u : 0u;
+            uint64_t* done_bar = &bar_done[rd];
+            if (elect_one()) {
+              mma(d_tmem, a, bd, acc0);
+              mma(d_tmem, a + 8, bd + 2, 1u);
+              mma(d_tmem, a + 16, bd + 4, 1u);
+              mma(d_tmem, a + 24, bd + 6, 1u);
+              commit(done_bar);
+            }
+            __syncwarp();
+            if (++xs == SX) xs = 0;
+            if (++rd == RD) rd = 0;
+            if (++as_ == AS) {
+              as_ = 0;
+              a_par ^= 1u;
+            }
+          }
+          kt += nbs;
         }
-        kt += nbs;
-        g += nbs;
+        if (!live) break;
+        if (elect_one()) commit(&bar_accfull[ab]);
+        __syncwarp();
+        ++j;
       }
-      if (!live) break;
-      if (elect_one()) mma_commit(&bar_accfull[ab]);
+      if (elect_one()) {
+        if constexpr (PAIR)
+          mma_commit2_mc(&bar_drain, static_cast<uint16_t>(0x1));
+        else
+          mma_commit(&bar_drain);
+        volatile int no_abort = 0;
+        mbar_wait(&bar_drain, 0, &no_abort, p.err, kDevTimeoutDrain);
+      }
       __syncwarp();
-      ++j;
     }
-    if (elect_one()) {
-      mma_commit(&bar_drain);
-      volatile int no_abort = 0;
-      mbar_wait(&bar_drain, 0, &no_abort, p.err, kDevTimeoutDrain);
-    }
-    __syncwarp();
   } else if (warp < 6) {
     // ============================================================ epilogue
     // Per chunk of kEpiRows accumulator columns (output rows): (1) each thread
@@ -615,8 +693,8 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
       // one decision for all four warps: they meet at named barriers below
       if (!named_bar_and(1, 128, ready && !*abort_flag)) break;
       tc_fence_after();
-      const int nb = it.tile % p.num_nb;
-      const int64_t m0 = static_cast<int64_t>(it.tile / p.num_nb) * BN;
+      const int nb = tile_nb(it.tile);
+      const int64_t m0 = static_cast<int64_t>(tile_mb(it.tile)) * BN;
       const int nl = quad * 32 + lane;  // phase 1: weight column within the tile
       const int nn = nb * kWqNBlock + nl;
       const bool col_ok = nn < p.n;
@@ -667,7 +745,7 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
           // the whole accumulator is in registers or staged: hand it back
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&bar_accempty[ab]);
+          if (lane == 0) arrive_mma_cta(&bar_accempty[ab]);
         }
         if (part) {
 #pragma unroll
@@ -711,7 +789,7 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
     uint32_t g = 0;
     bool live = true;
     while (live && walk.next(p, it)) {
-      const int nb = it.tile % p.num_nb;
+      const int nb = tile_nb(it.tile);
       const int nn = nb * kWqNBlock + r;
       const bool col_ok = nn < p.n;
       ColConst cc{};
@@ -792,28 +870,76 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK>::kThreads, 1)
           live = false;
           break;
         }
-        if (lane == 0) mbar_arrive(&bar_afull[as]);
+        if (lane == 0) arrive_mma_cta(&bar_afull[as]);
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  // a pair tears down together: no arrival or commit may target an exited CTA
+  if constexpr (PAIR) cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::kTmemCols);
+    if constexpr (PAIR)
+      tmem_dealloc2(tmem, C::kTmemCols);
+    else
+      tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
-template <int BN, int DG, int WK, bool BF16>
+template <int BN, int DG, int WK, bool BF16, bool PAIR>
 cudaError_t launch_one(const CUtensorMap& tmap, const WqParams& p, int grid, cudaStream_t s) {
-  using C = Cfg<BN, DG, WK>;
-  auto kern = wqmm_tc_kernel<BN, DG, WK, BF16>;
+  using C = Cfg<BN, DG, WK, PAIR>;
+  auto kern = wqmm_tc_kernel<BN, DG, WK, BF16, PAIR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   if (grid <= 0) return cudaErrorInvalidConfiguration;
-  kern<<<static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, s>>>(tmap, p);
-  return cudaGetLastError();
+  if constexpr (!PAIR) {
+    kern<<<static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, s>>>(tmap, p);
+    return cudaGetLastError();
+  } else {
+    if (grid % 2 != 0) return cudaErrorInvalidConfiguration;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(C::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, tmap, p);
+  }
+}
+
+// Pairs of CTAs (clusters of two) that can be resident at once for this
+// configuration, or 0 if none.
+template <int BN, int DG, int WK, bool BF16>
+int pair_slots_one() {
+  using C = Cfg<BN, DG, WK, true>;
+  auto kern = wqmm_tc_kernel<BN, DG, WK, BF16, true>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
 }
 
 // dequantisation groups: small tiles have little MMA work per k step, so more
@@ -823,15 +949,17 @@ constexpr int dgroups() {
   return 4;
 }
 
-template <int BN>
+template <int BN, bool PAIR>
 cudaError_t launch_bn(const CUtensorMap& tmap, const WqParams& p, int wk, bool bf16, int grid, cudaStream_t s) {
   constexpr int DG = dgroups<BN>();
   if (wk == kW4)
-    return bf16 ? launch_one<BN, DG, kW4, true>(tmap, p, grid, s) : launch_one<BN, DG, kW4, false>(tmap, p, grid, s);
+    return bf16 ? launch_one<BN, DG, kW4, true, PAIR>(tmap, p, grid, s)
+                : launch_one<BN, DG, kW4, false, PAIR>(tmap, p, grid, s);
   if (wk == kW8)
-    return bf16 ? launch_one<BN, DG, kW8, true>(tmap, p, grid, s) : launch_one<BN, DG, kW8, false>(tmap, p, grid, s);
-  return bf16 ? launch_one<BN, DG, kWFp8, true>(tmap, p, grid, s)
-              : launch_one<BN, DG, kWFp8, false>(tmap, p, grid, s);
+    return bf16 ? launch_one<BN, DG, kW8, true, PAIR>(tmap, p, grid, s)
+                : launch_one<BN, DG, kW8, false, PAIR>(tmap, p, grid, s);
+  return bf16 ? launch_one<BN, DG, kWFp8, true, PAIR>(tmap, p, grid, s)
+              : launch_one<BN, DG, kWFp8, false, PAIR>(tmap, p, grid, s);
 }
 
 // ---------------------------------------------------------------- stream-K fix-up
@@ -879,15 +1007,27 @@ int wqmm_ctas_per_sm(int bn, int wk) {
   return 1;  // every configuration uses most of the SM's shared memory for its ring
 }
 
+int wqmm_pair_slots(int bn, int wk, bool act_bf16) {
+  if (bn != 192) return 0;  // CTA pairs are built for the 192-row m tile
+  constexpr int DG = dgroups<192>();
+  if (wk == kW4) return act_bf16 ? pair_slots_one<192, DG, kW4, true>() : pair_slots_one<192, DG, kW4, false>();
+  if (wk == kW8) return act_bf16 ? pair_slots_one<192, DG, kW8, true>() : pair_slots_one<192, DG, kW8, false>();
+  return act_bf16 ? pair_slots_one<192, DG, kWFp8, true>() : pair_slots_one<192, DG, kWFp8, false>();
+}
+
 cudaError_t launch_wqmm_gemm(const CUtensorMap& tmap_x1, const WqParams& p, int bn, int wk, bool act_bf16,
                              int grid, cudaStream_t s) {
+  if (p.pair) {
+    if (bn != 192) return cudaErrorInvalidValue;
+    return launch_bn<192, true>(tmap_x1, p, wk, act_bf16, grid, s);
+  }
   switch (bn) {
-    case 16: return launch_bn<16>(tmap_x1, p, wk, act_bf16, grid, s);
-    case 32: return launch_bn<32>(tmap_x1, p, wk, act_bf16, grid, s);
-    case 64: return launch_bn<64>(tmap_x1, p, wk, act_bf16, grid, s);
-    case 128: return launch_bn<128>(tmap_x1, p, wk, act_bf16, grid, s);
-    case 192: return launch_bn<192>(tmap_x1, p, wk, act_bf16, grid, s);
-    case 256: return launch_bn<256>(tmap_x1, p, wk, act_bf16, grid, s);
+    case 16: return launch_bn<16, false>(tmap_x1, p, wk, act_bf16, grid, s);
+    case 32: return launch_bn<32, false>(tmap_x1, p, wk, act_bf16, grid, s);
+    case 64: return launch_bn<64, false>(tmap_x1, p, wk, act_bf16, grid, s);
+    case 128: return launch_bn<128, false>(tmap_x1, p, wk, act_bf16, grid, s);
+    case 192: return launch_bn<192, false>(tmap_x1, p, wk, act_bf16, grid, s);
+    case 256: return launch_bn<256, false>(tmap_x1, p, wk, act_bf16, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }
