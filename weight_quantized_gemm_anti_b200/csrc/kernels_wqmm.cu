@@ -295,14 +295,37 @@ struct GroupRow {
     row = hidx / gq;
     rem = hidx - row * gq;
   }
-  __device__ __forceinline__ void advance(int halves, int gq) {
-    rem += halves;
-    while (rem >= gq) {
+  // advance by q * gq + rq halves (q, rq precomputed once: rq < gq)
+  __device__ __forceinline__ void advance(int q, int rq, int gq) {
+    row += q;
+    rem += rq;
+    if (rem >= gq) {
       rem -= gq;
       ++row;
     }
   }
   __device__ __forceinline__ int row1(int gq) const { return row + (rem + 1 >= gq ? 1 : 0); }
+};
+
+// Position in a ring of N slots (and its phase parity) of the k steps one
+// dequantisation group handles: they are D apart, so the position advances by
+// a compile-time stride instead of being recomputed by division.
+template <uint32_t N, uint32_t D>
+struct Cursor {
+  uint32_t i, ph;
+  __device__ __forceinline__ void init(uint32_t v) {
+    i = v % N;
+    ph = (v / N) & 1u;
+  }
+  __device__ __forceinline__ void adv() {
+    uint32_t j = i + D % N;
+    ph ^= (D / N) & 1u;
+    if (j >= N) {
+      j -= N;
+      ph ^= 1u;
+    }
+    i = j;
+  }
 };
 
 __device__ __forceinline__ GroupSO load_group_so(const WqParams& p, int kt, const GroupRow& gr, int gq, int nn,
@@ -786,9 +809,29 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR>::kThreads, 1)
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
     const bool grp = (p.mode == kPerGroup);
     const int gq = grp ? p.group_size / 32 : 1;   // 32-wide halves per group
-    uint32_t g = 0;
+    // This group's k steps are g = dg, dg + DG, dg + 2 DG, ... of the CTA's
+    // walk; the ring positions of step g advance by DG steps each time.
+    constexpr int Q = C::kWQ;
+    static_assert(DG % Q == 0 || Q % DG == 0, "weight stage granularity");
+    constexpr uint32_t kWAdv = DG >= Q ? DG / Q : 1;  // weight stages per own step (Q <= DG)
+    static_assert(DG >= Q, "a dequantisation group takes whole weight stages");
+    Cursor<SW, kWAdv> wcur;            // weight stage of step g
+    Cursor<AS, DG> acur;               // A stage of step g
+    Cursor<SX, DG> xcur;               // x1 slab of step g
+    Cursor<RD, DG> dcur;               // done barrier of step g - AS (valid once g >= AS)
+    wcur.init(static_cast<uint32_t>(dg) / Q);
+    acur.init(static_cast<uint32_t>(dg));
+    xcur.init(static_cast<uint32_t>(dg));
+    dcur.init(static_cast<uint32_t>(dg) + RD - AS);  // phase flipped: (g - AS) / RD = (g - AS + RD) / RD - 1
+    const uint32_t wslot = static_cast<uint32_t>(dg) % Q;  // slot of step g inside its weight stage
+    // group rows advance by 2 DG halves per own step
+    const int gadv_q = grp ? (2 * DG) / gq : 0;
+    const int gadv_r = grp ? (2 * DG) - gadv_q * gq : 0;
+    uint32_t g = static_cast<uint32_t>(dg);  // this group's next k step
+    uint32_t gbase = 0;                      // step index of the current item's first k step
     bool live = true;
     while (live && walk.next(p, it)) {
+      const int len = it.kt1 - it.kt0;
       const int nb = tile_nb(it.tile);
       const int nn = nb * kWqNBlock + r;
       const bool col_ok = nn < p.n;
@@ -796,30 +839,29 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR>::kThreads, 1)
       if (!grp) cc = col_const<BF16, WK>(p, nn, col_ok);
       // per-group scale/offset come straight from global memory (L2), one of
       // this group's k steps ahead of their use
-      const int kt_first = it.kt0 + static_cast<int>((dg - static_cast<int>(g % DG) + DG) % DG);
       GroupRow grow{};
       GroupSO so_next{};
-      if (grp && kt_first < it.kt1) {
+      if (grp && g - gbase < static_cast<uint32_t>(len)) {
+        const int kt_first = it.kt0 + static_cast<int>(g - gbase);
         grow.init(2 * kt_first, gq);
         so_next = load_group_so(p, kt_first, grow, gq, nn, col_ok);
       }
-      for (int kt = it.kt0; kt < it.kt1; ++kt, ++g) {
-        if (static_cast<int>(g % DG) != dg) continue;
+      for (; g - gbase < static_cast<uint32_t>(len); g += DG) {
+        const int kt = it.kt0 + static_cast<int>(g - gbase);
         const GroupSO so = so_next;
         if (grp && kt + DG < it.kt1) {
-          grow.advance(2 * DG, gq);
+          grow.advance(gadv_q, gadv_r, gq);
           so_next = load_group_so(p, kt + DG, grow, gq, nn, col_ok);
         }
-        const int sw = (g / C::kWQ) % SW;
-        const int as = g % AS;
+        const int sw = static_cast<int>(wcur.i);
+        const int as = static_cast<int>(acur.i);
         // 1) weight tile -> registers, then hand the stage back to the producer
-        bool got = mbar_wait_sleep(&bar_wfull[sw], (g / C::kWQ / SW) & 1, abort_flag, p.err, kDevTimeoutDequant,
-                                   32, 256);
+        bool got = mbar_wait_sleep(&bar_wfull[sw], wcur.ph, abort_flag, p.err, kDevTimeoutDequant, 32, 256);
         if (!__all_sync(kFull, got)) {
           live = false;
           break;
         }
-        const uint8_t* wt = s_w + sw * C::kWStageBytes + (g % C::kWQ) * kTile;
+        const uint8_t* wt = s_w + sw * C::kWStageBytes + wslot * kTile;
         constexpr int kChunks = (WK == kW4) ? 2 : 4;
         uint4 ch[kChunks];
 #pragma unroll
@@ -855,8 +897,8 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR>::kThreads, 1)
           for (int c = 0; c < 4; ++c) dq_fp8<BF16>(ch[c], a + 8 * c);
         }
         // 3) the A stage is free once the MMA of step g - AS is done
-        got = g < static_cast<uint32_t>(AS) ||
-              mbar_wait(&bar_done[(g - AS) % RD], ((g - AS) / RD) & 1, abort_flag, p.err, kDevTimeoutDequant);
+        got = g < static_cast<uint32_t>(AS) || mbar_wait(&bar_done[dcur.i], dcur.ph ^ 1u, abort_flag, p.err,
+                                                         kDevTimeoutDequant);
         if (!__all_sync(kFull, got)) {  // tcgen05.st below is warp-collective
           live = false;
           break;
@@ -865,13 +907,18 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR>::kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         // 4) the stage may be issued once this step's x1 slab has landed too
-        got = mbar_wait(&bar_xfull[g % SX], (g / SX) & 1, abort_flag, p.err, kDevTimeoutDequant);
+        got = mbar_wait(&bar_xfull[xcur.i], xcur.ph, abort_flag, p.err, kDevTimeoutDequant);
         if (!__all_sync(kFull, got)) {
           live = false;
           break;
         }
         if (lane == 0) arrive_mma_cta(&bar_afull[as]);
+        wcur.adv();
+        acur.adv();
+        xcur.adv();
+        dcur.adv();
       }
+      gbase += static_cast<uint32_t>(len);
     }
   }
 
