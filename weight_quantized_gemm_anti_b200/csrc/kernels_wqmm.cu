@@ -284,6 +284,7 @@ __device__ __forceinline__ void dq8_group_half(const uint4 chA, const uint4 chB,
 // (per-group mode).
 struct GroupSO {
   uint16_t s[2], o[2];
+  bool one_row;  // warp-uniform: both halves use the same group row (and lie inside k)
 };
 
 // Group row of half index hidx = 2*kt (+1 for the second half): row = hidx / gq,
@@ -332,6 +333,7 @@ __device__ __forceinline__ GroupSO load_group_so(const WqParams& p, int kt, cons
                                                  bool col_ok) {
   GroupSO r;
   const int rows[2] = {gr.row, gr.row1(gq)};
+  r.one_row = rows[0] == rows[1] && kt * kWqKTile + 32 < p.k;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const bool use = col_ok && (kt * kWqKTile + 32 * h < p.k);
@@ -405,7 +407,9 @@ __device__ __forceinline__ ColConst col_const(const WqParams& p, int nn, bool co
   return c;
 }
 
-template <int BN, int DG, int WK, bool BF16, bool PAIR>
+// GRP: per-group scale/offset (compile-time, so each kernel carries the code of
+// its own mode only)
+template <int BN, int DG, int WK, bool BF16, bool PAIR, bool GRP>
 __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR>::kThreads, 1)
     wqmm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x1, const WqParams p) {
   using C = Cfg<BN, DG, WK, PAIR>;
@@ -728,7 +732,7 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR>::kThreads, 1)
 #pragma unroll
       for (int i = 0; i < 8; ++i) bias8[i] = 0.f;
       if (it.slot < 0) {
-        if (p.mode != kPerGroup) {
+        if constexpr (!GRP) {
           const ColConst cc = col_const<BF16, WK>(p, nn, col_ok);
           escale = (WK == kWFp8 || cc.fast) ? cc.s : 1.f;
         }
@@ -807,7 +811,7 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR>::kThreads, 1)
     const int quad = warp & 3;                    // TMEM lane quadrant this warp may access
     const int r = quad * 32 + lane;               // weight column within the 128-column block
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
-    const bool grp = (p.mode == kPerGroup);
+    constexpr bool grp = GRP;
     const int gq = grp ? p.group_size / 32 : 1;   // 32-wide halves per group
     // This group's k steps are g = dg, dg + DG, dg + 2 DG, ... of the CTA's
     // walk; the ring positions of step g advance by DG steps each time.
@@ -871,9 +875,18 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR>::kThreads, 1)
         // 2) dequantise in registers: needs nothing but the weights
         uint32_t a[32];
         if constexpr (WK == kW4) {
-          if (grp) {
-            dq4_group_half<BF16, 0>(ch[0], so.s[0], so.o[0], a);
-            dq4_group_half<BF16, 1>(ch[1], so.s[1], so.o[1], a);
+          if constexpr (GRP) {
+            const float off = act_f32(so.o[0], BF16);
+            if (so.one_row && __all_sync(kFull, small_int(off))) {
+              // one group row for the whole step: its constants once
+              const float c = off - (BF16 ? 136.f : 1032.f);
+              const uint32_t c2 = pack2<BF16>(c, c), s2 = splat_bits(so.s[0]);
+              dq4_fast<BF16, true>(ch[0], c2, s2, a);
+              dq4_fast<BF16, true>(ch[1], c2, s2, a + 16);
+            } else {
+              dq4_group_half<BF16, 0>(ch[0], so.s[0], so.o[0], a);
+              dq4_group_half<BF16, 1>(ch[1], so.s[1], so.o[1], a);
+            }
           } else if (cc.fast) {
             dq4_fast<BF16, false>(ch[0], cc.c2, 0u, a);
             dq4_fast<BF16, false>(ch[1], cc.c2, 0u, a + 16);
@@ -882,7 +895,7 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR>::kThreads, 1)
             dq4_general<BF16>(ch[1], cc.off, cc.s, a + 16);
           }
         } else if constexpr (WK == kW8) {
-          if (grp) {
+          if constexpr (GRP) {
             dq8_group_half<BF16, 0>(ch[0], ch[1], so.s[0], so.o[0], a);
             dq8_group_half<BF16, 1>(ch[2], ch[3], so.s[1], so.o[1], a);
           } else if (cc.fast) {
@@ -935,10 +948,10 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR>::kThreads, 1)
   }
 }
 
-template <int BN, int DG, int WK, bool BF16, bool PAIR>
+template <int BN, int DG, int WK, bool BF16, bool PAIR, bool GRP>
 cudaError_t launch_one(const CUtensorMap& tmap, const WqParams& p, int grid, cudaStream_t s) {
   using C = Cfg<BN, DG, WK, PAIR>;
-  auto kern = wqmm_tc_kernel<BN, DG, WK, BF16, PAIR>;
+  auto kern = wqmm_tc_kernel<BN, DG, WK, BF16, PAIR, GRP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   if (grid <= 0) return cudaErrorInvalidConfiguration;
@@ -968,7 +981,7 @@ cudaError_t launch_one(const CUtensorMap& tmap, const WqParams& p, int grid, cud
 template <int BN, int DG, int WK, bool BF16>
 int pair_slots_one() {
   using C = Cfg<BN, DG, WK, true>;
-  auto kern = wqmm_tc_kernel<BN, DG, WK, BF16, true>;
+  auto kern = wqmm_tc_kernel<BN, DG, WK, BF16, true, (WK != kWFp8)>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess) return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2, 1, 1);
@@ -996,17 +1009,25 @@ constexpr int dgroups() {
   return 4;
 }
 
+template <int BN, bool PAIR, int WK, bool BF16>
+cudaError_t launch_mode(const CUtensorMap& tmap, const WqParams& p, int grid, cudaStream_t s) {
+  constexpr int DG = dgroups<BN>();
+  if constexpr (WK == kWFp8) {  // fp8 weights have per-channel scales only
+    return launch_one<BN, DG, WK, BF16, PAIR, false>(tmap, p, grid, s);
+  } else {
+    return p.mode == kPerGroup ? launch_one<BN, DG, WK, BF16, PAIR, true>(tmap, p, grid, s)
+                               : launch_one<BN, DG, WK, BF16, PAIR, false>(tmap, p, grid, s);
+  }
+}
+
 template <int BN, bool PAIR>
 cudaError_t launch_bn(const CUtensorMap& tmap, const WqParams& p, int wk, bool bf16, int grid, cudaStream_t s) {
-  constexpr int DG = dgroups<BN>();
   if (wk == kW4)
-    return bf16 ? launch_one<BN, DG, kW4, true, PAIR>(tmap, p, grid, s)
-                : launch_one<BN, DG, kW4, false, PAIR>(tmap, p, grid, s);
+    return bf16 ? launch_mode<BN, PAIR, kW4, true>(tmap, p, grid, s) : launch_mode<BN, PAIR, kW4, false>(tmap, p, grid, s);
   if (wk == kW8)
-    return bf16 ? launch_one<BN, DG, kW8, true, PAIR>(tmap, p, grid, s)
-                : launch_one<BN, DG, kW8, false, PAIR>(tmap, p, grid, s);
-  return bf16 ? launch_one<BN, DG, kWFp8, true, PAIR>(tmap, p, grid, s)
-              : launch_one<BN, DG, kWFp8, false, PAIR>(tmap, p, grid, s);
+    return bf16 ? launch_mode<BN, PAIR, kW8, true>(tmap, p, grid, s) : launch_mode<BN, PAIR, kW8, false>(tmap, p, grid, s);
+  return bf16 ? launch_mode<BN, PAIR, kWFp8, true>(tmap, p, grid, s)
+              : launch_mode<BN, PAIR, kWFp8, false>(tmap, p, grid, s);
 }
 
 // ---------------------------------------------------------------- stream-K fix-up
