@@ -149,6 +149,36 @@ def test_wqmm_cta_pair_parity(spec, whole_tiles):
     check_wqmm(case)
 
 
+# Whole tiles on single CTAs (m > 128: 128- and 192-row m tiles): with an even
+# number of k steps the dequantisation groups take turns of two k steps (their
+# per-turn waits, bookkeeping and scale/offset loads shared); with an odd number
+# they take one step per turn.
+WHOLE = [
+    ("whole_i4_g128_bf16", (400, 1024), 256, "bf16", "i4", "group", 128, {"scale_range": (0.005, 0.05),
+                                                                          "offset_range": (-4, 4)}),
+    ("whole_i4_g32_bf16", (300, 512), 384, "bf16", "i4", "group", 32, {}),
+    ("whole_i4_g96_f16_rows_straddle", (200, 768), 256, "f16", "i4", "group", 96, {}),
+    ("whole_i4_g64_bf16_fractional", (257, 512), 128, "bf16", "i4", "group", 64, {"fractional_offset": True}),
+    ("whole_i4_chan_bf16_odd_ksteps", (300, 320), 256, "bf16", "i4", "channel", 0, {}),
+    ("whole_i8_tensor_bf16_x3", (330, 640), 192, "bf16", "i8", "tensor", 0, {"scale_const": 0.01,
+                                                                             "offset_const": 3.0}),
+    ("whole_i8_g64_f16", (140, 256), 160, "f16", "i8", "group", 64, {}),
+    ("whole_i8_chan_bf16_k_ragged", (200, 352), 96, "bf16", "i8", "channel", 0, {}),
+    ("whole_fp8_chan_bf16", (150, 512), 128, "bf16", "fp8", "channel", 0, {"offset": False}),
+    ("whole_i4_g128_bf16_bn128", (100, 512), 256, "bf16", "i4", "group", 128, {}),
+]
+
+
+@pytest.mark.parametrize("spec", WHOLE, ids=[s[0] for s in WHOLE])
+def test_wqmm_whole_tiles_parity(spec, monkeypatch):
+    monkeypatch.setenv("WQMM_STREAMK", "0")
+    monkeypatch.setenv("WQMM_PAIR", "0")
+    name, x1s, n, act, wdt, mode, G, extra = spec
+    case = WL.make_wqmm_case(name=name, x1_shape=x1s, n=n, act=act, wdt=wdt, mode=mode, group_size=G,
+                             seed=zlib.crc32(name.encode()) % 10000, **extra)
+    check_wqmm(case)
+
+
 def test_wqmm_cta_pair_matches_single_cta(monkeypatch):
     # the same problem with and without CTA pairs: both within tolerance of the
     # oracle, and close to each other

@@ -59,7 +59,10 @@ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 
 constexpr int cmax(int a, int b) { return a > b ? a : b; }
 
-template <int BN, int DG, int WK, bool PAIR = false>
+// SPG: k steps a dequantisation group takes per turn (1 or 2); a group's
+// per-turn costs (barrier waits, loop and ring bookkeeping, scale/offset
+// loads) are shared by its SPG steps.
+template <int BN, int DG, int WK, bool PAIR = false, int SPG = 1>
 struct Cfg {
   static constexpr int kTile = wq_tile_bytes(WK);
   // x1 slab of one k step held by this CTA: BN rows, or BN / 2 when a CTA pair
@@ -68,9 +71,9 @@ struct Cfg {
   static constexpr int kAccCols = BN < 32 ? 32 : BN;
   static constexpr int kNAcc = (2 * kAccCols + 4 * 32 <= 512) ? 2 : 1;
   static constexpr int kACol0 = kNAcc * kAccCols;
-  // TMEM A stages: as many as fit (up to 12), a multiple of DG so that every
-  // dequantisation group owns its own stages
-  static constexpr int kAStages = cmin(12, (512 - kACol0) / 32 / DG * DG);
+  // TMEM A stages: as many as fit (up to 12), a multiple of DG * SPG so that
+  // every dequantisation group owns its own stages
+  static constexpr int kAStages = cmin(12, (512 - kACol0) / 32 / (DG * SPG) * (DG * SPG));
   static constexpr int kTmemCols = pow2ceil(kACol0 + kAStages * 32);
   // shared memory: a weight ring (read by the dequantisers, released as soon
   // as a tile is in registers) and an x1 ring (read by the MMA).  An x1 slab is
@@ -100,7 +103,8 @@ struct Cfg {
   static constexpr int kXWarp2 = 7 + 4 * DG;
   static constexpr int kThreads = 32 * (8 + 4 * DG);
   static constexpr int kSmemBytes = kXStages * kX1Bytes + kWStages * kWStageBytes + kStageBytes + 1024;
-  static_assert(kAStages >= DG && kAStages % DG == 0, "A stages");
+  static_assert(kAStages >= DG * SPG && kAStages % (DG * SPG) == 0, "A stages");
+  static_assert(kWQ % SPG == 0 && (DG * SPG) % kWQ == 0, "a group's turn lies in one weight stage; turns cover whole stages");
   static_assert(kACol0 + kAStages * 32 <= 512, "TMEM budget");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   static_assert(kXStages >= 2 * kBatch && kAStages >= 2 * kBatch, "a batch must fit twice in each ring");
@@ -344,6 +348,42 @@ __device__ __forceinline__ GroupSO load_group_so(const WqParams& p, int kt, cons
   return r;
 }
 
+// Scale/offset bits of one column for the NH 32-wide halves of one turn of a
+// dequantisation group (NH = 2 SPG), per-group mode.
+template <int NH>
+struct GroupSOn {
+  uint16_t s[NH], o[NH];
+  bool one_row;  // warp-uniform: all halves use the same group row and lie inside k
+};
+
+template <int NH>
+__device__ __forceinline__ GroupSOn<NH> load_group_son(const WqParams& p, int kt, const GroupRow& gr, int gq, int nn,
+                                                       bool col_ok) {
+  GroupSOn<NH> r;
+  int rows[NH];
+  int row = gr.row, rem = gr.rem;
+  rows[0] = row;
+#pragma unroll
+  for (int h = 1; h < NH; ++h) {
+    if (++rem >= gq) {
+      rem -= gq;
+      ++row;
+    }
+    rows[h] = row;
+  }
+  r.one_row = rows[NH - 1] == rows[0] && kt * kWqKTile + 32 * (NH - 1) < p.k;
+  // every half loads (predicated, no branch): loads behind a branch issue late
+  // and their latency shows
+#pragma unroll
+  for (int h = 0; h < NH; ++h) {
+    const bool use = col_ok && (kt * kWqKTile + 32 * h < p.k);
+    const int64_t idx = static_cast<int64_t>(rows[h]) * p.n + nn;
+    r.s[h] = use ? __ldg(p.scale + idx) : uint16_t(0);
+    r.o[h] = (use && p.offset) ? __ldg(p.offset + idx) : uint16_t(0);
+  }
+  return r;
+}
+
 // ---------------------------------------------------------------- schedule
 struct Item {
   int tile, kt0, kt1, slot;  // slot < 0: whole tile, write the output
@@ -409,10 +449,10 @@ __device__ __forceinline__ ColConst col_const(const WqParams& p, int nn, bool co
 
 // GRP: per-group scale/offset (compile-time, so each kernel carries the code of
 // its own mode only)
-template <int BN, int DG, int WK, bool BF16, bool PAIR, bool GRP>
-__global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR>::kThreads, 1)
+template <int BN, int DG, int WK, bool BF16, bool PAIR, bool GRP, int SPG>
+__global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR, SPG>::kThreads, 1)
     wqmm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x1, const WqParams p) {
-  using C = Cfg<BN, DG, WK, PAIR>;
+  using C = Cfg<BN, DG, WK, PAIR, SPG>;
   constexpr int SX = C::kXStages;
   constexpr int SW = C::kWStages;
   constexpr int AS = C::kAStages;
@@ -454,7 +494,7 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR>::kThreads, 1)
     }
     for (int i = 0; i < SW; ++i) {
       mbar_init(&bar_wfull[i], 1);
-      mbar_init(&bar_wempty[i], 4 * C::kWQ);
+      mbar_init(&bar_wempty[i], 4 * C::kWQ / SPG);
     }
     for (int i = 0; i < AS; ++i) {
       mbar_init(&bar_afull[i], kArrivers);
@@ -813,26 +853,26 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR>::kThreads, 1)
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
     constexpr bool grp = GRP;
     const int gq = grp ? p.group_size / 32 : 1;   // 32-wide halves per group
-    // This group's k steps are g = dg, dg + DG, dg + 2 DG, ... of the CTA's
-    // walk; the ring positions of step g advance by DG steps each time.
+    // Group dg takes turns of SPG consecutive k steps: its turns start at
+    // g = SPG * dg, SPG * (dg + DG), ... of the CTA's walk, so every ring
+    // position advances by CYC = DG * SPG steps per turn.  (With SPG = 2 the
+    // launcher guarantees that a turn never spans two tiles.)
     constexpr int Q = C::kWQ;
-    static_assert(DG % Q == 0 || Q % DG == 0, "weight stage granularity");
-    constexpr uint32_t kWAdv = DG >= Q ? DG / Q : 1;  // weight stages per own step (Q <= DG)
-    static_assert(DG >= Q, "a dequantisation group takes whole weight stages");
-    Cursor<SW, kWAdv> wcur;            // weight stage of step g
-    Cursor<AS, DG> acur;               // A stage of step g
-    Cursor<SX, DG> xcur;               // x1 slab of step g
-    Cursor<RD, DG> dcur;               // done barrier of step g - AS (valid once g >= AS)
-    wcur.init(static_cast<uint32_t>(dg) / Q);
-    acur.init(static_cast<uint32_t>(dg));
-    xcur.init(static_cast<uint32_t>(dg));
-    dcur.init(static_cast<uint32_t>(dg) + RD - AS);  // phase flipped: (g - AS) / RD = (g - AS + RD) / RD - 1
-    const uint32_t wslot = static_cast<uint32_t>(dg) % Q;  // slot of step g inside its weight stage
-    // group rows advance by 2 DG halves per own step
-    const int gadv_q = grp ? (2 * DG) / gq : 0;
-    const int gadv_r = grp ? (2 * DG) - gadv_q * gq : 0;
-    uint32_t g = static_cast<uint32_t>(dg);  // this group's next k step
-    uint32_t gbase = 0;                      // step index of the current item's first k step
+    constexpr uint32_t CYC = DG * SPG;
+    constexpr int NH = 2 * SPG;  // 32-wide halves of a turn
+    Cursor<SW, CYC / Q> wcur;    // weight stage of the turn
+    Cursor<AS, CYC> acur;        // A stage of the turn's first step
+    Cursor<SX, CYC> xcur;        // x1 slab of the turn's first step
+    Cursor<RD, CYC> dcur;        // done barrier of the turn's last step - AS (valid once that is >= 0)
+    wcur.init(static_cast<uint32_t>(SPG * dg) / Q);
+    acur.init(static_cast<uint32_t>(SPG * dg));
+    xcur.init(static_cast<uint32_t>(SPG * dg));
+    dcur.init(static_cast<uint32_t>(SPG * dg + SPG - 1) + RD - AS);  // phase flipped
+    const uint32_t wslot = static_cast<uint32_t>(SPG * dg) % Q;      // first slot of the turn in its stage
+    const int gadv_q = grp ? static_cast<int>(2 * CYC) / gq : 0;     // group rows per turn
+    const int gadv_r = grp ? static_cast<int>(2 * CYC) - gadv_q * gq : 0;
+    uint32_t g = static_cast<uint32_t>(SPG * dg);  // first k step of this group's next turn
+    uint32_t gbase = 0;                             // step index of the current item's first k step
     bool live = true;
     while (live && walk.next(p, it)) {
       const int len = it.kt1 - it.kt0;
@@ -841,91 +881,118 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR>::kThreads, 1)
       const bool col_ok = nn < p.n;
       ColConst cc{};
       if (!grp) cc = col_const<BF16, WK>(p, nn, col_ok);
-      // per-group scale/offset come straight from global memory (L2), one of
-      // this group's k steps ahead of their use
+      // per-group scale/offset come straight from global memory (L2), one turn
+      // ahead of their use
       GroupRow grow{};
-      GroupSO so_next{};
+      GroupSOn<NH> so_next{};
       if (grp && g - gbase < static_cast<uint32_t>(len)) {
         const int kt_first = it.kt0 + static_cast<int>(g - gbase);
         grow.init(2 * kt_first, gq);
-        so_next = load_group_so(p, kt_first, grow, gq, nn, col_ok);
+        so_next = load_group_son<NH>(p, kt_first, grow, gq, nn, col_ok);
       }
-      for (; g - gbase < static_cast<uint32_t>(len); g += DG) {
+      for (; g - gbase < static_cast<uint32_t>(len); g += CYC) {
         const int kt = it.kt0 + static_cast<int>(g - gbase);
-        const GroupSO so = so_next;
-        if (grp && kt + DG < it.kt1) {
+        const GroupSOn<NH> so = so_next;
+        if (grp && kt + static_cast<int>(CYC) < it.kt1) {
           grow.advance(gadv_q, gadv_r, gq);
-          so_next = load_group_so(p, kt + DG, grow, gq, nn, col_ok);
+          so_next = load_group_son<NH>(p, kt + CYC, grow, gq, nn, col_ok);
         }
         const int sw = static_cast<int>(wcur.i);
-        const int as = static_cast<int>(acur.i);
-        // 1) weight tile -> registers, then hand the stage back to the producer
+        // 1) the turn's weight tiles -> registers, then hand the stage back
         bool got = mbar_wait_sleep(&bar_wfull[sw], wcur.ph, abort_flag, p.err, kDevTimeoutDequant, 32, 256);
         if (!__all_sync(kFull, got)) {
           live = false;
           break;
         }
-        const uint8_t* wt = s_w + sw * C::kWStageBytes + wslot * kTile;
         constexpr int kChunks = (WK == kW4) ? 2 : 4;
-        uint4 ch[kChunks];
+        uint4 ch[SPG][kChunks];
 #pragma unroll
-        for (int c = 0; c < kChunks; ++c) ch[c] = *reinterpret_cast<const uint4*>(wt + (c * kWqNBlock + r) * 16);
+        for (int j = 0; j < SPG; ++j) {
+          const uint8_t* wt = s_w + sw * C::kWStageBytes + (wslot + j) * kTile;
+#pragma unroll
+          for (int c = 0; c < kChunks; ++c) ch[j][c] = *reinterpret_cast<const uint4*>(wt + (c * kWqNBlock + r) * 16);
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar_wempty[sw]);
-        // 2) dequantise in registers: needs nothing but the weights
-        uint32_t a[32];
-        if constexpr (WK == kW4) {
-          if constexpr (GRP) {
-            const float off = act_f32(so.o[0], BF16);
-            if (so.one_row && __all_sync(kFull, small_int(off))) {
-              // one group row for the whole step: its constants once
-              const float c = off - (BF16 ? 136.f : 1032.f);
-              const uint32_t c2 = pack2<BF16>(c, c), s2 = splat_bits(so.s[0]);
-              dq4_fast<BF16, true>(ch[0], c2, s2, a);
-              dq4_fast<BF16, true>(ch[1], c2, s2, a + 16);
-            } else {
-              dq4_group_half<BF16, 0>(ch[0], so.s[0], so.o[0], a);
-              dq4_group_half<BF16, 1>(ch[1], so.s[1], so.o[1], a);
-            }
-          } else if (cc.fast) {
-            dq4_fast<BF16, false>(ch[0], cc.c2, 0u, a);
-            dq4_fast<BF16, false>(ch[1], cc.c2, 0u, a + 16);
-          } else {
-            dq4_general<BF16>(ch[0], cc.off, cc.s, a);
-            dq4_general<BF16>(ch[1], cc.off, cc.s, a + 16);
-          }
-        } else if constexpr (WK == kW8) {
-          if constexpr (GRP) {
-            dq8_group_half<BF16, 0>(ch[0], ch[1], so.s[0], so.o[0], a);
-            dq8_group_half<BF16, 1>(ch[2], ch[3], so.s[1], so.o[1], a);
-          } else if (cc.fast) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) dq8_fast<BF16, false>(ch[c], cc.off, cc.s, cc.c2, 0u, a + 8 * c);
-          } else {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) dq8_general<BF16>(ch[c], cc.off, cc.s, a + 8 * c);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) dq_fp8<BF16>(ch[c], a + 8 * c);
+        // per-group int4 with one group row for the whole turn: constants once
+        bool row_fast = false;
+        uint32_t rc2 = 0, rs2 = 0;
+        if constexpr (GRP && WK == kW4) {
+          const float off = act_f32(so.o[0], BF16);
+          row_fast = so.one_row && __all_sync(kFull, small_int(off));
+          const float c = off - (BF16 ? 136.f : 1032.f);
+          rc2 = pack2<BF16>(c, c);
+          rs2 = splat_bits(so.s[0]);
         }
-        // 3) the A stage is free once the MMA of step g - AS is done
-        got = g < static_cast<uint32_t>(AS) || mbar_wait(&bar_done[dcur.i], dcur.ph ^ 1u, abort_flag, p.err,
-                                                         kDevTimeoutDequant);
-        if (!__all_sync(kFull, got)) {  // tcgen05.st below is warp-collective
+#pragma unroll
+        for (int j = 0; j < SPG; ++j) {
+          // 2) dequantise step j in registers: needs nothing but the weights
+          uint32_t a[32];
+          if constexpr (WK == kW4) {
+            if constexpr (GRP) {
+              if (row_fast) {
+                dq4_fast<BF16, true>(ch[j][0], rc2, rs2, a);
+                dq4_fast<BF16, true>(ch[j][1], rc2, rs2, a + 16);
+              } else {
+                dq4_group_half<BF16, 0>(ch[j][0], so.s[2 * j], so.o[2 * j], a);
+                dq4_group_half<BF16, 1>(ch[j][1], so.s[2 * j + 1], so.o[2 * j + 1], a);
+              }
+            } else if (cc.fast) {
+              dq4_fast<BF16, false>(ch[j][0], cc.c2, 0u, a);
+              dq4_fast<BF16, false>(ch[j][1], cc.c2, 0u, a + 16);
+            } else {
+              dq4_general<BF16>(ch[j][0], cc.off, cc.s, a);
+              dq4_general<BF16>(ch[j][1], cc.off, cc.s, a + 16);
+            }
+          } else if constexpr (WK == kW8) {
+            if constexpr (GRP) {
+              dq8_group_half<BF16, 0>(ch[j][0], ch[j][1], so.s[2 * j], so.o[2 * j], a);
+              dq8_group_half<BF16, 1>(ch[j][2], ch[j][3], so.s[2 * j + 1], so.o[2 * j + 1], a);
+            } else if (cc.fast) {
+#pragma unroll
+              for (int c = 0; c < 4; ++c) dq8_fast<BF16, false>(ch[j][c], cc.off, cc.s, cc.c2, 0u, a + 8 * c);
+            } else {
+#pragma unroll
+              for (int c = 0; c < 4; ++c) dq8_general<BF16>(ch[j][c], cc.off, cc.s, a + 8 * c);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) dq_fp8<BF16>(ch[j][c], a + 8 * c);
+          }
+          if (j == 0) {
+            // 3) the turn's A stages are free once the MMA of its last step -
+            // AS is done (MMAs complete in order, so that covers every step)
+            got = g + SPG - 1 < static_cast<uint32_t>(AS) ||
+                  mbar_wait(&bar_done[dcur.i], dcur.ph ^ 1u, abort_flag, p.err, kDevTimeoutDequant);
+            got = __all_sync(kFull, got);  // tcgen05.st below is warp-collective
+            if (!got) break;
+          }
+          tmem_st_x32(tmem + lane_addr + C::kACol0 + (acur.i + j) * 32, a);
+        }
+        if (!got) {
           live = false;
           break;
         }
-        tmem_st_x32(tmem + lane_addr + C::kACol0 + as * 32, a);
         tmem_wait_st();
         tc_fence_before();
-        // 4) the stage may be issued once this step's x1 slab has landed too
-        got = mbar_wait(&bar_xfull[xcur.i], xcur.ph, abort_flag, p.err, kDevTimeoutDequant);
+        // 4) each step may be issued once its x1 slab has landed too
+#pragma unroll
+        for (int j = 0; j < SPG; ++j) {
+          uint32_t xi = xcur.i + j, xph = xcur.ph;
+          if (xi >= static_cast<uint32_t>(SX)) {
+            xi -= SX;
+            xph ^= 1u;
+          }
+          got = got && mbar_wait(&bar_xfull[xi], xph, abort_flag, p.err, kDevTimeoutDequant);
+        }
         if (!__all_sync(kFull, got)) {
           live = false;
           break;
         }
-        if (lane == 0) arrive_mma_cta(&bar_afull[as]);
+        if (lane == 0) {
+#pragma unroll
+          for (int j = 0; j < SPG; ++j) arrive_mma_cta(&bar_afull[acur.i + j]);
+        }
         wcur.adv();
         acur.adv();
         xcur.adv();
@@ -948,10 +1015,10 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR>::kThreads, 1)
   }
 }
 
-template <int BN, int DG, int WK, bool BF16, bool PAIR, bool GRP>
+template <int BN, int DG, int WK, bool BF16, bool PAIR, bool GRP, int SPG>
 cudaError_t launch_one(const CUtensorMap& tmap, const WqParams& p, int grid, cudaStream_t s) {
-  using C = Cfg<BN, DG, WK, PAIR>;
-  auto kern = wqmm_tc_kernel<BN, DG, WK, BF16, PAIR, GRP>;
+  using C = Cfg<BN, DG, WK, PAIR, SPG>;
+  auto kern = wqmm_tc_kernel<BN, DG, WK, BF16, PAIR, GRP, SPG>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   if (grid <= 0) return cudaErrorInvalidConfiguration;
@@ -981,7 +1048,7 @@ cudaError_t launch_one(const CUtensorMap& tmap, const WqParams& p, int grid, cud
 template <int BN, int DG, int WK, bool BF16>
 int pair_slots_one() {
   using C = Cfg<BN, DG, WK, true>;
-  auto kern = wqmm_tc_kernel<BN, DG, WK, BF16, true, (WK != kWFp8)>;
+  auto kern = wqmm_tc_kernel<BN, DG, WK, BF16, true, (WK != kWFp8), 1>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess) return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2, 1, 1);
@@ -1009,15 +1076,26 @@ constexpr int dgroups() {
   return 4;
 }
 
+// Turns of two k steps per dequantisation group (two groups) for wide m
+// tiles over whole tiles with an even number of k steps; one step per turn
+// (four groups) otherwise.
+template <int BN, bool PAIR, int WK, bool BF16, int SPG>
+cudaError_t launch_spg(const CUtensorMap& tmap, const WqParams& p, int grid, cudaStream_t s) {
+  constexpr int DG = SPG == 2 ? 2 : dgroups<BN>();
+  if constexpr (WK == kWFp8) {  // fp8 weights have per-channel scales only
+    return launch_one<BN, DG, WK, BF16, PAIR, false, SPG>(tmap, p, grid, s);
+  } else {
+    return p.mode == kPerGroup ? launch_one<BN, DG, WK, BF16, PAIR, true, SPG>(tmap, p, grid, s)
+                               : launch_one<BN, DG, WK, BF16, PAIR, false, SPG>(tmap, p, grid, s);
+  }
+}
+
 template <int BN, bool PAIR, int WK, bool BF16>
 cudaError_t launch_mode(const CUtensorMap& tmap, const WqParams& p, int grid, cudaStream_t s) {
-  constexpr int DG = dgroups<BN>();
-  if constexpr (WK == kWFp8) {  // fp8 weights have per-channel scales only
-    return launch_one<BN, DG, WK, BF16, PAIR, false>(tmap, p, grid, s);
-  } else {
-    return p.mode == kPerGroup ? launch_one<BN, DG, WK, BF16, PAIR, true>(tmap, p, grid, s)
-                               : launch_one<BN, DG, WK, BF16, PAIR, false>(tmap, p, grid, s);
+  if constexpr (BN >= 128 && !PAIR) {
+    if (!p.stream_k && p.kt_total % 2 == 0) return launch_spg<BN, PAIR, WK, BF16, 2>(tmap, p, grid, s);
   }
+  return launch_spg<BN, PAIR, WK, BF16, 1>(tmap, p, grid, s);
 }
 
 template <int BN, bool PAIR>
