@@ -316,6 +316,34 @@ def test_qmm_small_parity_and_exact_accumulator(spec):
     assert rel_err(g, ye) <= TOL[out]
 
 
+# Clusters of two CTAs share each int8 MMA (M = 256 rows of x1, 128 per CTA;
+# each CTA loads half of the 256-column weight tile).  WQMM_PAIR=1 selects it at
+# any size; odd 128-row block counts leave the second CTA of the last pair
+# without rows (its loads are zero-filled and its outputs masked).
+QPAIR = [
+    ("qp_bf16_odd_blocks", (300, 384), 512, "bf16", {}),
+    ("qp_f16_no_pertoken", (256, 256), 256, "f16", {"pertoken": False}),
+    ("qp_bf16_3d_no_bias_x3", (2, 200, 1024), 768, "bf16", {"bias": False, "x3": False}),
+    ("qp_bf16_tensor_dq", (129, 128), 256, "bf16", {"dq_per_tensor": True}),
+]
+
+
+@pytest.mark.parametrize("spec", QPAIR, ids=[s[0] for s in QPAIR])
+def test_qmm_cta_pair_parity_and_exact_accumulator(spec, monkeypatch):
+    monkeypatch.setenv("WQMM_PAIR", "1")
+    name, x1s, n, out, extra = spec
+    case = WL.make_qmm_case(name=name, x1_shape=x1s, n=n, out=out, seed=zlib.crc32(name.encode()) % 1000, **extra)
+    d = C.qmm_to_device(case)
+    acc = torch.empty((case.m, n), dtype=torch.int32, device="cuda")
+    C.qmm_call(d, raw_acc=acc)
+    torch.cuda.synchronize()
+    no_device_error()
+    a_ref, ye, _ = oracle.qmm(case)
+    assert np.array_equal(acc.cpu().numpy(), a_ref)
+    g = dec(gpu_bits(d.out), out)
+    assert rel_err(g, ye) <= TOL[out]
+
+
 def test_qmm_transposed_weight_and_unpacked():
     case = WL.make_qmm_case(x1_shape=(40, 128), n=96, x2_transposed=True, seed=12)
     d = C.qmm_to_device(case, pack=False)

@@ -175,6 +175,24 @@ int sm_count() {
 
 uint64_t round_up(uint64_t v, uint64_t a) { return (v + a - 1) / a * a; }
 
+// Resident CTA pairs of the pair-mode int8 GEMM per (device, output type).
+int qmm_pair_slots_cached(bool out_bf16) {
+  static std::mutex mu;
+  static std::map<std::pair<int, int>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  const auto key = std::make_pair(dev, out_bf16 ? 1 : 0);
+  std::lock_guard<std::mutex> lock(mu);
+  auto f = cache.find(key);
+  if (f != cache.end()) return f->second;
+  const int v = qmm_pair_slots(out_bf16);
+  cache[key] = v;
+  return v;
+}
+
 // Resident CTA pairs of the pair-mode GEMM, per (device, m tile, weight kind,
 // activation type); 0 when there is no pair mode or no device.
 int pair_slots(int bn, int wk, bool bf16) {
@@ -616,9 +634,11 @@ EncodeFn encode_fn() {
 }
 
 // 2-D row-major matrix (rows x cols elements of `esize` bytes), box (box_cols x
-// box_rows), 128-byte swizzle, out-of-bounds elements read as zero.
+// box_rows), 128-byte swizzle unless told otherwise, out-of-bounds elements
+// read as zero.
 wqmm_status make_tmap(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int esize, int64_t rows,
-                      int64_t cols, int box_cols, int box_rows) {
+                      int64_t cols, int box_cols, int box_rows,
+                      CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeFn fn = encode_fn();
   if (!fn) return fail(WQMM_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
@@ -626,7 +646,7 @@ wqmm_status make_tmap(CUtensorMap* map, const void* base, CUtensorMapDataType dt
   cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(WQMM_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
   return WQMM_SUCCESS;
 }
@@ -803,7 +823,27 @@ wqmm_status run_qmm(void* ws, wqmm_executor* ex, cudaStream_t s) {
   p.dq_bf16 = ex->dq_dtype == WQMM_DT_BF16;
   p.dq_per_tensor = ex->dq_per_tensor;
   p.out_bf16 = ex->act_dtype == WQMM_DT_BF16;
-  e = launch_qmm_gemm(tmap, p, s);
+  // enough 256-row tiles for every pair of SMs: clusters of two CTAs share
+  // each MMA, so each SM loads half of the weight tile (WQMM_PAIR=0 turns it off)
+  p.pair_grid = 0;
+  {
+    const char* pair_env = std::getenv("WQMM_PAIR");
+    const bool forbid_pair = pair_env && std::atoi(pair_env) == 0;
+    const bool force_pair = pair_env && std::atoi(pair_env) == 1;  // tests: pairs at any size
+    const int64_t ptiles = static_cast<int64_t>((p.num_mb + 1) / 2) * p.num_nb;
+    const int slots = forbid_pair ? 0 : qmm_pair_slots_cached(p.out_bf16 != 0);
+    if (slots > 0 && (ptiles >= slots || force_pair)) p.pair_grid = static_cast<int>(2 * (ptiles < slots ? ptiles : slots));
+  }
+  CUtensorMap tmap_w = tmap;
+  if (p.pair_grid > 0) {
+    // the packed weight is already in the shared-memory (swizzled) order: a
+    // plain 2-D view, 128-byte rows, each CTA of a pair copying 128 of them
+    const int64_t rows = static_cast<int64_t>(p.num_nb) * p.kt_total * kQNBlock;
+    st = make_tmap(&tmap_w, wpack, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows, kQKTile, kQKTile, kQNBlock / 2,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st) return st;
+  }
+  e = launch_qmm_gemm(tmap, tmap_w, p, s);
   if (e != cudaSuccess) return cuda_fail(e, "int8 GEMM launch");
   return WQMM_SUCCESS;
 }

@@ -93,6 +93,7 @@ struct QParams {
   int dq_bf16;                 // 1: bf16 dequant scale, 0: f32
   int dq_per_tensor;           // 1: dq has one element
   int out_bf16;                // 1: bf16 output, 0: f16
+  int pair_grid;               // > 0: clusters of two CTAs share each MMA (tiles of 256 rows); grid size
 };
 
 struct PackParams {
@@ -132,7 +133,12 @@ cudaError_t launch_wqmm_gemm(const CUtensorMap& tmap_x1, const WqParams& p, int 
                              int grid, cudaStream_t s);
 cudaError_t launch_wqmm_fixup(const FixupParams& p, cudaStream_t s);
 cudaError_t launch_wqmm_epilogue(const EpiParams& p, cudaStream_t s);
-cudaError_t launch_qmm_gemm(const CUtensorMap& tmap_x1, const QParams& p, cudaStream_t s);
+// tmap_w: the packed int8 weight viewed as rows of 128 bytes (box 128 x 128,
+// no swizzle), used by the pair mode only.
+cudaError_t launch_qmm_gemm(const CUtensorMap& tmap_x1, const CUtensorMap& tmap_w, const QParams& p,
+                            cudaStream_t s);
+// Clusters of two CTAs of the pair-mode int8 GEMM that fit at once (0 if none).
+int qmm_pair_slots(bool out_bf16);
 
 // Device error word of the library (first kernel error code, 0 if none).
 uint32_t* device_error_word();
