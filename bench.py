@@ -70,6 +70,38 @@ def load_traffic(workload: str):
     return e.get("dram_bytes_per_launch")
 
 
+# ------------------------------------------------------------------ schedule
+def wqmm_schedule(m: int, n: int, k: int, sms: int) -> dict:
+    """The anti-quant GEMM's schedule as the library's phase 1 chooses it with
+    no tuning overrides (a restatement of its planner, checked against the
+    library's workspace sizes in the CPU tests): m tile, stream-K or whole
+    tiles, and whether a fix-up kernel follows the GEMM."""
+    bn = 16 if m <= 16 else 32 if m <= 32 else 64 if m <= 64 else 128 if m <= 128 else 256
+    num_nb = -(-n // 128)
+    kt = -(-k // 64)
+    tiles = -(-m // bn) * num_nb
+    out = {"bn": bn, "stream_k": False, "inline": False, "partial_bytes": 0, "flag_bytes": 0}
+    if k == 0 or kt < 2:
+        return out
+    rem = tiles % sms
+    if tiles < sms:
+        dp = 0
+    elif bn < 128 and rem > 0 and rem * 100 <= 85 * sms:
+        dp = tiles - rem
+    else:
+        return out
+    unit = 2 if (bn >= 128 and kt % 2 == 0) else 1
+    split = tiles - dp
+    T = split * kt // unit
+    grid = sms if dp > 0 else min(T, sms)
+    skg = min(T, grid)
+    owner = lambda s: ((s + 1) * skg - 1) // T
+    ms = max(owner((r * kt + kt - 1) // unit) - owner(r * kt // unit) + 1 for r in range(split))
+    out.update(stream_k=True, inline=ms <= 4, partial_bytes=split * ms * bn * 128 * 4,
+               flag_bytes=split * ms * 8 if ms <= 4 else 0)
+    return out
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     def __init__(self):
@@ -184,8 +216,13 @@ class Problem:
         if self.int8:
             return 1
         c = self.case
-        # mirror of the library's split-K choice, read back from a planned executor
-        return 1 + (1 if self.ws_size > 0 else 0)
+        k = c.k
+        m = 1
+        for d in c.x1_shape[:-1]:
+            m *= d
+        sched = wqmm_schedule(m, c.n, k, self.torch.cuda.get_device_properties(0).multi_processor_count)
+        # the GEMM, plus the fix-up kernel when split tiles are reduced by one
+        return 1 + (1 if sched["stream_k"] and not sched["inline"] else 0)
 
 
 def time_device(prob: Problem, steps: int, warmup: int, flush_bytes: int):

@@ -234,3 +234,29 @@ def test_pack_size_queries():
     assert st == W.SUCCESS and nb == 2 * 2 * 8192                                   # 2 n-blocks x 2 k-tiles, padded
     st, _ = W.wqmm_pack_weight_size(T((64, 128), W.DT_F16))
     assert st == W.ERR_PARAM_INVALID
+
+
+# ------------------------------------------------------------------ schedule
+@pytest.mark.parametrize("m,k,n", [
+    (4096, 4096, 4096),    # whole tiles (CTA pairs for int4): no workspace
+    (2048, 4096, 4096),    # whole tiles
+    (16, 8192, 28672),     # narrow tiles, last wave split, owners reduce inline
+    (40, 512, 21760),      # 170 tiles: 148 whole + 22 split
+    (16, 4096, 256),       # 2 tiles over many CTAs: fix-up kernel
+    (300, 512, 256),       # wide tiles, fewer than the CTAs: two-step units
+    (200, 448, 384),       # odd k-step count
+])
+def test_schedule_mirror_matches_library_workspace(m, k, n):
+    import bench
+    st, ws = wq(x1=((m, k), W.DT_BF16), x2=((k, n), W.DT_I4), scale=((n,), None), x2_fmt=W.FORMAT_PACKED)
+    assert st == W.SUCCESS
+    sms = 148  # phase 1 without a GPU plans for a B200
+    try:
+        import torch
+        if torch.cuda.is_available():
+            sms = torch.cuda.get_device_properties(0).multi_processor_count
+    except ImportError:
+        pass
+    s = bench.wqmm_schedule(m, n, k, sms)
+    rnd = lambda b: -(-b // 256) * 256
+    assert ws == rnd(s["partial_bytes"]) + rnd(s["flag_bytes"]), (s, ws)

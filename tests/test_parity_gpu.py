@@ -118,7 +118,7 @@ def test_wqmm_small_parity(spec):
 
 
 # ---------------------------------------------------------------- CTA pairs
-# m > 128 selects the 192-row m tile; with whole tiles per CTA (stream-K off)
+# With the 192- or 256-row m tile (WQMM_BN), whole tiles per CTA (stream-K off)
 # and WQMM_PAIR=1, two CTAs of a cluster share each MMA (cta_group::2), each
 # holding half of the x1 slab and its own 128 weight columns.  Odd column-block counts leave
 # the second CTA of the last pair without weights (its outputs are masked).
@@ -134,10 +134,11 @@ PAIRS = [
 ]
 
 
-@pytest.fixture
-def whole_tiles(monkeypatch):
+@pytest.fixture(params=["192", "256"])
+def whole_tiles(request, monkeypatch):
     monkeypatch.setenv("WQMM_STREAMK", "0")
     monkeypatch.setenv("WQMM_PAIR", "1")
+    monkeypatch.setenv("WQMM_BN", request.param)  # the m tiles CTA pairs are built for
     yield
 
 
@@ -169,14 +170,77 @@ WHOLE = [
 ]
 
 
+@pytest.mark.parametrize("bn", ["192", "256"])
 @pytest.mark.parametrize("spec", WHOLE, ids=[s[0] for s in WHOLE])
-def test_wqmm_whole_tiles_parity(spec, monkeypatch):
+def test_wqmm_whole_tiles_parity(spec, bn, monkeypatch):
     monkeypatch.setenv("WQMM_STREAMK", "0")
     monkeypatch.setenv("WQMM_PAIR", "0")
+    if spec[1][0] > 128:  # the m tile of wide problems: two TMEM accumulators (192) or one (256)
+        monkeypatch.setenv("WQMM_BN", bn)
     name, x1s, n, act, wdt, mode, G, extra = spec
     case = WL.make_wqmm_case(name=name, x1_shape=x1s, n=n, act=act, wdt=wdt, mode=mode, group_size=G,
                              seed=zlib.crc32(name.encode()) % 10000, **extra)
     check_wqmm(case)
+
+
+# ---------------------------------------------------------------- split last wave
+# Narrow m tiles, more tiles than CTAs, the last wave partly filled: whole tiles
+# for the full waves, then the k steps of the remaining tiles split evenly over
+# the CTAs.  With at most four owners per split tile the owner of its first k
+# steps adds the others' partials itself (inline); with more, or with
+# WQMM_SK_INLINE=0, every owner writes a partial and the fix-up kernel reduces.
+# Wide tiles use stream-K only when there are fewer tiles than CTAs (then with
+# two-step units and two-step dequantisation turns).  WQMM_GRID shrinks the
+# persistent grid so that these schedules arise at sizes the oracle computes
+# quickly.
+# name, x1_shape, n, act, wdt, mode, G, extras, grid (None: all SMs), env
+HYBRID = [
+    # 18 tiles on 8 CTAs: 16 whole + 2 split four ways (inline)
+    ("hyb_i4_g64_bf16_m40", (40, 512), 2304, "bf16", "i4", "group", 64, {"scale_range": (0.005, 0.05),
+                                                                       "offset_range": (-4, 4)}, 8, {}),
+    ("hyb_i4_g64_bf16_m40_fixup", (40, 512), 2304, "bf16", "i4", "group", 64, {}, 8, {"WQMM_SK_INLINE": "0"}),
+    ("hyb_i8_chan_f16_m16", (16, 640), 1280, "f16", "i8", "channel", 0, {}, 4, {}),
+    ("hyb_i4_g128_bf16_m64_bias_x3", (64, 1024), 1152, "bf16", "i4", "group", 128, {}, 4, {}),
+    ("hyb_fp8_chan_bf16_m32", (32, 512), 640, "bf16", "fp8", "channel", 0, {"offset": False}, 2, {}),
+    ("hyb_i8_tensor_bf16_m24_x3", (24, 640), 768, "bf16", "i8", "tensor", 0, {"scale_const": 0.01,
+                                                                              "offset_const": 3.0}, 4, {}),
+    # one split tile over eight owners: the fix-up kernel
+    ("hyb_i8_g32_bf16_m20_eight_owners", (20, 1024), 1152, "bf16", "i8", "group", 32, {}, 8, {}),
+    # wide tiles, fewer tiles than CTAs: every tile split (two-step units), inline
+    ("sk_wide_i4_g128_bf16", (300, 512), 256, "bf16", "i4", "group", 128, {}, None, {}),
+    ("sk_wide_i8_chan_f16_odd_ksteps", (200, 448), 384, "f16", "i8", "channel", 0, {}, None, {}),
+]
+
+
+@pytest.mark.parametrize("spec", HYBRID, ids=[s[0] for s in HYBRID])
+def test_wqmm_split_last_wave_parity(spec, monkeypatch):
+    name, x1s, n, act, wdt, mode, G, extra, grid, env = spec
+    if grid:
+        monkeypatch.setenv("WQMM_GRID", str(grid))
+    monkeypatch.setenv("WQMM_PAIR", "0")
+    for key, val in env.items():
+        monkeypatch.setenv(key, val)
+    case = WL.make_wqmm_case(name=name, x1_shape=x1s, n=n, act=act, wdt=wdt, mode=mode, group_size=G,
+                             seed=zlib.crc32(name.encode()) % 10000, **extra)
+    d = C.wqmm_to_device(case)
+    ws = C.wqmm_call(d)
+    torch.cuda.synchronize()
+    no_device_error()
+    assert ws is not None and ws.numel() > 0, "a stream-K plan keeps fp32 partials in the workspace"
+    first = gpu_bits(d.out)
+    ye, _ = oracle.wqmm(case)
+    g = dec(first, case.act)
+    assert np.isfinite(g).all()
+    assert rel_err(g, ye) <= TOL[case.act], f"{name}: rel err {rel_err(g, ye):.3e}"
+    # a second run repeats every bit (the fix-up sums partials in a fixed order)
+    C.wqmm_call(d, workspace=ws)
+    torch.cuda.synchronize()
+    no_device_error()
+    assert np.array_equal(first, gpu_bits(d.out)), f"{name}: repeated runs differ"
+    # and whole tiles on the same grid agree within the tolerance
+    monkeypatch.setenv("WQMM_STREAMK", "0")
+    whole = dec(run_wqmm(case), case.act)
+    assert rel_err(g, whole) <= TOL[case.act]
 
 
 def test_wqmm_cta_pair_matches_single_cta(monkeypatch):
@@ -184,6 +248,7 @@ def test_wqmm_cta_pair_matches_single_cta(monkeypatch):
     # oracle, and close to each other
     monkeypatch.setenv("WQMM_STREAMK", "0")
     monkeypatch.setenv("WQMM_PAIR", "1")
+    monkeypatch.setenv("WQMM_BN", "192")
     case = WL.make_wqmm_case(name="pair_vs_single", x1_shape=(512, 1024), n=512, act="bf16", wdt="i4", mode="group",
                              group_size=128, scale_range=(0.005, 0.05), offset_range=(-4, 4), seed=11)
     a = dec(run_wqmm(case), case.act)

@@ -3,6 +3,7 @@
 // -> CheckShape, "返回值与错误码"), launch planning, one-shot executors, and
 // phase-2 launches on the caller's stream.  Phase 1 is host-only: it makes no
 // CUDA call except an optional SM-count query used to size split-K.
+#include <atomic>
 #include <chrono>
 #include <cstdarg>
 #include <cstdio>
@@ -18,11 +19,16 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <unistd.h>
 
 #include "../../include/wqmm.h"
 #include "internal.h"
 
 using namespace wqmm;
+
+namespace wqmm {
+thread_local uint64_t g_plan_ws_cap = 0;
+}  // namespace wqmm
 
 namespace {
 
@@ -70,7 +76,7 @@ struct wqmm_executor {
   const void* bias = nullptr;
   const void* x3 = nullptr;
   uint64_t workspace = 0;
-  Region ws_pack, ws_scale, ws_offset, ws_partial;
+  Region ws_pack, ws_scale, ws_offset, ws_partial, ws_flags;
   // wqmm
   const void* scale = nullptr;
   const void* offset = nullptr;
@@ -80,7 +86,11 @@ struct wqmm_executor {
   int num_groups = 0;
   int bn = 256;
   int grid = 1;        // persistent CTAs of the GEMM
-  int stream_k = 0;    // 1: k steps of all tiles split evenly over the grid, partials + fix-up
+  int stream_k = 0;    // 1: stream-K -- the k steps of tiles dp_tiles.. split evenly over the grid, partials + fix-up
+  int dp_tiles = 0;    // stream-K: tiles run whole before the split ones (a multiple of the grid)
+  int sk_unit = 1;     // stream-K: split granularity in k steps
+  int sk_grid = 0;     // stream-K: CTAs sharing the split tiles
+  int sk_inline = 0;   // stream-K: the first owner of a split tile reduces it (no fix-up kernel)
   int pair = 0;        // 1: clusters of two CTAs share each MMA (256 weight columns per pair tile)
   int num_pnb = 0;     // pair: 256-column blocks
   int num_tiles = 0;
@@ -156,6 +166,23 @@ wqmm_status check_descriptor(const wqmm_tensor* t, const char* name) {
   if (t->format != WQMM_FORMAT_ND && t->format != WQMM_FORMAT_PACKED)
     return fail(WQMM_ERR_PARAM_INVALID, "%s: unknown format %d", name, t->format);
   return WQMM_SUCCESS;
+}
+
+// A value no earlier launch has written into a stream-K flag: a process-wide
+// counter (odd values, step 2) started at a value mixed from the clocks and the
+// process id, so that flags left in reused memory (by this or an earlier
+// process) do not match.
+uint64_t next_launch_token() {
+  static std::atomic<uint64_t> counter{[] {
+    uint64_t x = static_cast<uint64_t>(std::chrono::steady_clock::now().time_since_epoch().count());
+    x ^= static_cast<uint64_t>(std::chrono::system_clock::now().time_since_epoch().count()) << 21;
+    x ^= static_cast<uint64_t>(getpid()) << 40;
+    x ^= x >> 33;
+    x *= 0xff51afd7ed558ccdULL;
+    x ^= x >> 33;
+    return x | 1ULL;
+  }()};
+  return counter.fetch_add(2, std::memory_order_relaxed);  // odd, never zero, never repeated
 }
 
 int sm_count() {
@@ -427,9 +454,9 @@ extern "C" wqmm_status wqmm_get_workspace_size(const wqmm_tensor* x1, const wqmm
   ex->num_groups = static_cast<int>(ng);
   uint64_t ws = 0;
   if (k > 0) {
-    // m tile: the smallest supported width that covers m; large m uses 192
-    // (two TMEM accumulators fit, so the epilogue overlaps the next tile)
-    ex->bn = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <= 128 ? 128 : 192;
+    // m tile: the smallest supported width that covers m; larger m uses 256,
+    // the widest MMA (the most MMA work per dequantised weight step)
+    ex->bn = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <= 128 ? 128 : 256;
     if (const char* env = std::getenv("WQMM_BN")) {  // tuning override
       const int v = std::atoi(env);
       if (v == 16 || v == 32 || v == 64 || v == 128 || v == 192 || v == 256) ex->bn = v;
@@ -442,33 +469,68 @@ extern "C" wqmm_status wqmm_get_workspace_size(const wqmm_tensor* x1, const wqmm
       delete ex;
       return fail(WQMM_ERR_INNER_TILING, "too many output tiles");
     }
-    const int64_t slots = static_cast<int64_t>(sm_count()) * wqmm_ctas_per_sm(ex->bn, 0);
+    int64_t slots = static_cast<int64_t>(sm_count()) * wqmm_ctas_per_sm(ex->bn, 0);
+    if (const char* env = std::getenv("WQMM_GRID")) {  // testing override: fewer persistent CTAs
+      const int64_t v = std::atoll(env);
+      if (v >= 1 && v < slots) slots = v;
+    }
     ex->num_tiles = static_cast<int>(tiles);
     ex->stream_k = 0;
+    ex->dp_tiles = 0;
     ex->grid = static_cast<int>(tiles < slots ? tiles : slots);
     const char* sk_env = std::getenv("WQMM_STREAMK");
     const bool force_sk = sk_env && std::atoi(sk_env) == 1;
     const bool forbid_sk = sk_env && std::atoi(sk_env) == 0;
-    if (!forbid_sk && (force_sk || tiles < slots) && kt >= 2) {
-      // fewer tiles than SMs: spread all k steps evenly over one CTA per SM
-      ex->stream_k = 1;
-      const int64_t total = tiles * kt;
-      ex->grid = static_cast<int>(total < slots ? total : slots);
-      int ms = 1;
-      for (int64_t t = 0; t < tiles; ++t) {
-        const int64_t c = sk_owner(t * kt + kt - 1, total, ex->grid) - sk_owner(t * kt, total, ex->grid) + 1;
-        if (c > ms) ms = static_cast<int>(c);
-      }
-      ex->max_slots = ms;
+    // Stream-K: with fewer tiles than CTAs, the k steps of all tiles are spread
+    // evenly over the CTAs.  With more, narrow m tiles (< 128 rows) run the whole
+    // waves as whole tiles and split a last, partly filled wave (at most 85%
+    // full) the same way over every CTA, so that no SM idles while others finish
+    // it.  (Measured on B200, wide tiles gain less from the split than its
+    // partial tiles cost.)  Splits fall on pairs of k steps when the
+    // dequantisers take two-step turns.
+    const int64_t rem = tiles % slots;
+    int64_t dp = -1;  // tiles run whole before the split ones; -1: no stream-K
+    if (!forbid_sk && kt >= 2) {
+      if (force_sk || tiles < slots)
+        dp = 0;
+      else if (ex->bn < 128 && rem > 0 && rem * 100 <= 85 * slots)
+        dp = tiles - rem;
     }
-    // 192-row m tiles over whole tiles can run as clusters of two CTAs that
-    // share each MMA (each CTA holds half of the x1 slab).  Measured on B200 it
-    // is not faster than single CTAs (both are bound by instruction issue in the
-    // dequantisation), so it is opt-in: WQMM_PAIR=1.
+    if (dp >= 0) {
+      const int unit = (ex->bn >= 128 && kt % 2 == 0) ? 2 : 1;
+      const int64_t split = tiles - dp;
+      const int64_t T = split * kt / unit;
+      const int64_t grid = dp > 0 ? slots : (T < slots ? T : slots);
+      const int64_t sk_grid = T < grid ? T : grid;  // every sharing CTA gets at least one unit
+      int ms = 1;
+      for (int64_t r = 0; r < split; ++r) {
+        const SkOwners o = sk_tile_owners(r, static_cast<int>(kt), unit, T, sk_grid);
+        if (o.last - o.first + 1 > ms) ms = static_cast<int>(o.last - o.first + 1);
+      }
+      const uint64_t partial_bytes = static_cast<uint64_t>(split) * ms * ex->bn * kWqNBlock * 4;
+      if (!(dp > 0 && g_plan_ws_cap > 0 && partial_bytes > g_plan_ws_cap)) {
+        ex->stream_k = 1;
+        ex->dp_tiles = static_cast<int>(dp);
+        ex->sk_unit = unit;
+        ex->sk_grid = static_cast<int>(sk_grid);
+        ex->grid = static_cast<int>(grid);
+        ex->max_slots = ms;
+        // a few owners per tile: the first owner, which reaches its part last,
+        // adds the others' partials itself; many: a fix-up kernel spreads the sums
+        ex->sk_inline = ms <= 4 ? 1 : 0;
+        if (const char* env = std::getenv("WQMM_SK_INLINE")) ex->sk_inline = (std::atoi(env) == 1 && ms <= 4) ? 1 : 0;
+      }
+    }
+    // 192- and 256-row m tiles over whole tiles can run as clusters of two CTAs
+    // that share each MMA (each CTA holds half of the x1 slab, so the x1 ring
+    // and the MMA issuer's batches are twice as deep).  Measured on B200 the
+    // 256-row pairs are faster for int4 weights (W4A16 g128 4096^3: 137.7 vs
+    // 141.3 us) and not for int8 (W8A16 2048x4096x4096: 94.3 vs 92.2 us): the
+    // default for int4 at 256 rows; WQMM_PAIR=1 / 0 forces them on / off.
     const char* pair_env = std::getenv("WQMM_PAIR");
-    const bool want_pair = pair_env && std::atoi(pair_env) == 1;
-    if (!ex->stream_k && want_pair && ex->bn == 192 && num_nb >= 2) {
-      const int wk = x2->dtype == WQMM_DT_I4 ? kW4 : (x2->dtype == WQMM_DT_I8 ? kW8 : kWFp8);
+    const int wk = x2->dtype == WQMM_DT_I4 ? kW4 : (x2->dtype == WQMM_DT_I8 ? kW8 : kWFp8);
+    const bool want_pair = pair_env ? std::atoi(pair_env) == 1 : (ex->bn == 256 && wk == kW4);
+    if (!ex->stream_k && want_pair && (ex->bn == 192 || ex->bn == 256) && num_nb >= 2) {
       const int ps = pair_slots(ex->bn, wk, adt == WQMM_DT_BF16);
       if (ps > 0) {
         const int64_t pnb = (num_nb + 1) / 2;
@@ -492,8 +554,12 @@ extern "C" wqmm_status wqmm_get_workspace_size(const wqmm_tensor* x1, const wqmm
       }
     }
     if (ex->stream_k) {
-      ex->ws_partial = {ws, static_cast<uint64_t>(tiles) * ex->max_slots * ex->bn * kWqNBlock * 4};
+      ex->ws_partial = {ws, static_cast<uint64_t>(tiles - ex->dp_tiles) * ex->max_slots * ex->bn * kWqNBlock * 4};
       ws = round_up(ws + ex->ws_partial.bytes, 256);
+      if (ex->sk_inline) {
+        ex->ws_flags = {ws, static_cast<uint64_t>(tiles - ex->dp_tiles) * ex->max_slots * 8};
+        ws = round_up(ws + ex->ws_flags.bytes, 256);
+      }
     }
   }
   ex->workspace = ws;
@@ -754,13 +820,19 @@ wqmm_status run_wqmm(void* ws, wqmm_executor* ex, cudaStream_t s) {
   p.pair = ex->pair;
   p.num_pnb = ex->num_pnb;
   p.stream_k = ex->stream_k;
+  p.dp_tiles = ex->dp_tiles;
+  p.sk_unit = ex->sk_unit;
+  p.sk_grid = ex->sk_grid;
+  p.sk_inline = ex->sk_inline;
+  p.sk_flags = ex->sk_inline ? reinterpret_cast<uint64_t*>(wsb + ex->ws_flags.offset) : nullptr;
+  p.sk_token = ex->sk_inline ? next_launch_token() : 0;
   p.max_slots = ex->max_slots;
   p.mode = ex->mode;
   p.group_size = ex->group_size;
   p.num_groups = ex->num_groups;
   e = launch_wqmm_gemm(tmap, p, ex->bn, wk, bf16, ex->grid, s);
   if (e != cudaSuccess) return cuda_fail(e, "anti-quant GEMM launch");
-  if (ex->stream_k) {
+  if (ex->stream_k && !ex->sk_inline) {
     FixupParams fp{};
     fp.partial = p.partial;
     fp.scale = scale;
@@ -773,8 +845,10 @@ wqmm_status run_wqmm(void* ws, wqmm_executor* ex, cudaStream_t s) {
     fp.bn = ex->bn;
     fp.num_nb = p.num_nb;
     fp.num_tiles = ex->num_tiles;
+    fp.dp_tiles = ex->dp_tiles;
     fp.kt_total = p.kt_total;
-    fp.grid = ex->grid;
+    fp.sk_unit = ex->sk_unit;
+    fp.sk_grid = ex->sk_grid;
     fp.max_slots = ex->max_slots;
     fp.mode = ex->mode;
     fp.act_bf16 = bf16;

@@ -32,7 +32,7 @@ struct WqParams {
   const uint16_t* bias;   // may be null
   const uint16_t* x3;     // may be null, (m, n)
   uint16_t* out;          // (m, n)
-  float* partial;         // stream-K partial tiles [num_tiles][max_slots][BN][128] fp32, or null
+  float* partial;         // stream-K partial tiles [num_tiles - dp_tiles][max_slots][BN][128] fp32, or null
   uint32_t* err;          // device error word
   int64_t m;
   int n, k;
@@ -44,18 +44,39 @@ struct WqParams {
                           // column blocks 2 * (t % num_pnb) + cluster rank)
   int pair;               // 1: clusters of two CTAs share each MMA (cta_group::2)
   int num_pnb;            // pair: ceil(num_nb / 2)
-  int stream_k;           // 0: whole tiles round-robin over the grid; 1: k-steps split evenly
-  int max_slots;          // stream-K: partial slots per tile
+  int stream_k;           // 0: whole tiles round-robin over the grid; 1: stream-K (below)
+  int dp_tiles;           // stream-K: tiles [0, dp_tiles) run whole, round-robin (a multiple of the grid);
+                          // the k steps of the tiles after them are split evenly over the grid
+  int sk_unit;            // stream-K: split points fall on multiples of this many k steps (1 or 2)
+  int sk_grid;            // stream-K: CTAs 0 .. sk_grid - 1 share the split tiles (each gets >= 1 unit)
+  int max_slots;          // stream-K: partial slots per split tile
+  int sk_inline;          // stream-K: 1 -- the owner of a split tile's first k steps (which it reaches
+                          // last) adds the other owners' partials and writes the output (no fix-up
+                          // kernel); 0 -- every owner writes a partial, the fix-up kernel reduces
+  uint64_t* sk_flags;     // stream-K inline: [num_tiles - dp_tiles][max_slots] "partial written" flags
+  uint64_t sk_token;      // stream-K inline: the value a flag holds once written in this launch
   int mode;               // QuantMode
   int group_size;         // per-group only
   int num_groups;         // rows of scale/offset in per-group mode
 };
 
-// Stream-K ownership: with T = num_tiles * kt_total k-steps split over G CTAs,
-// CTA c owns steps [floor(c*T/G), floor((c+1)*T/G)); the owner of step s is
-// floor(((s+1)*G - 1) / T).  Shared by the GEMM and the fix-up kernel.
+// Stream-K ownership: the k steps of the split tiles (tiles dp_tiles ..) are
+// counted in units of U steps from the first split tile; with T units split over
+// G CTAs, CTA c owns units [floor(c*T/G), floor((c+1)*T/G)); the owner of unit u
+// is floor(((u+1)*G - 1) / T).  Shared by the GEMM, the fix-up kernel and the
+// planner.
 __host__ __device__ inline int64_t sk_start(int64_t c, int64_t T, int64_t G) { return c * T / G; }
 __host__ __device__ inline int64_t sk_owner(int64_t s, int64_t T, int64_t G) { return ((s + 1) * G - 1) / T; }
+
+// CTAs holding a part of split tile r (0-based among the split tiles): first
+// and last owner.  A tile with a single owner is written whole by that CTA.
+struct SkOwners {
+  int64_t first, last;
+};
+__host__ __device__ inline SkOwners sk_tile_owners(int64_t r, int kt_total, int unit, int64_t T, int64_t G) {
+  const int64_t s0 = r * kt_total;
+  return {sk_owner(s0 / unit, T, G), sk_owner((s0 + kt_total - 1) / unit, T, G)};
+}
 
 struct FixupParams {      // stream-K reduction + epilogue
   const float* partial;
@@ -69,8 +90,10 @@ struct FixupParams {      // stream-K reduction + epilogue
   int bn;
   int num_nb;
   int num_tiles;
+  int dp_tiles;
   int kt_total;
-  int grid;
+  int sk_unit;
+  int sk_grid;
   int max_slots;
   int mode;
   int act_bf16;
@@ -145,5 +168,10 @@ uint32_t* device_error_word();
 
 // Set the calling thread's wqmm_last_error() message and return `code`.
 int32_t report_error(int32_t code, const char* msg);
+
+// Workspace ceiling for the planner on this thread (0: none): a stream-K split
+// of the last wave, which only saves time, is not planned when its partial
+// tiles would not fit.  Set around planning by callers with a fixed workspace.
+extern thread_local uint64_t g_plan_ws_cap;
 
 }  // namespace wqmm

@@ -387,42 +387,58 @@ __device__ __forceinline__ GroupSOn<NH> load_group_son(const WqParams& p, int kt
 // ---------------------------------------------------------------- schedule
 struct Item {
   int tile, kt0, kt1, slot;  // slot < 0: whole tile, write the output
+  int nadd;                  // > 0: this CTA finishes a split tile: add the partials of
+                             // slots 1 .. nadd (the other owners), write the output
 };
 
 // Identical walk of this CTA's work in every role.
+// The CTA's work items in order.  Whole tiles: tile = blockIdx.x, + grid, ...
+// (all tiles without stream-K; the first dp_tiles with it).  Stream-K: then
+// the CTA's even share of the k steps of the remaining tiles, cut at tile
+// boundaries; an item that is a part of a tile shared with other CTAs gets its
+// slot among the tile's owners (its fp32 partial goes to the fix-up kernel, or,
+// in inline mode, to the first owner, which adds them all and writes the
+// output); a tile the CTA owns alone is an ordinary whole tile (slot -1).
 struct Walker {
-  int64_t cur, end, T, step;
+  int64_t dcur, dend, step;  // whole tiles
+  int64_t cur, end, T;       // stream-K range, in k steps from the first split tile; T in units
   // pair: both CTAs of a pair walk the same pair tiles (no stream-K then)
   __device__ __forceinline__ void init(const WqParams& p, bool pair) {
+    dcur = pair ? (blockIdx.x >> 1) : blockIdx.x;
+    step = pair ? (gridDim.x >> 1) : gridDim.x;
     if (p.stream_k) {
-      T = static_cast<int64_t>(p.num_tiles) * p.kt_total;
-      cur = sk_start(blockIdx.x, T, gridDim.x);
-      end = sk_start(blockIdx.x + 1, T, gridDim.x);
-      step = gridDim.x;
+      dend = p.dp_tiles;
+      T = static_cast<int64_t>(p.num_tiles - p.dp_tiles) * p.kt_total / p.sk_unit;
+      const bool in_sk = static_cast<int>(blockIdx.x) < p.sk_grid;
+      cur = in_sk ? sk_start(blockIdx.x, T, p.sk_grid) * p.sk_unit : 0;
+      end = in_sk ? sk_start(blockIdx.x + 1, T, p.sk_grid) * p.sk_unit : 0;
     } else {
-      T = 0;
-      cur = pair ? (blockIdx.x >> 1) : blockIdx.x;
-      step = pair ? (gridDim.x >> 1) : gridDim.x;
-      end = p.num_tiles;
+      dend = p.num_tiles;
+      T = cur = end = 0;
     }
   }
   __device__ __forceinline__ bool next(const WqParams& p, Item& it) {
-    if (cur >= end) return false;
-    if (!p.stream_k) {
-      it.tile = static_cast<int>(cur);
+    if (dcur < dend) {
+      it.tile = static_cast<int>(dcur);
       it.kt0 = 0;
       it.kt1 = p.kt_total;
       it.slot = -1;
-      cur += step;
+      it.nadd = 0;
+      dcur += step;
       return true;
     }
-    const int64_t tile = cur / p.kt_total;
-    const int64_t tile_end = (tile + 1) * p.kt_total;
+    if (cur >= end) return false;
+    const int64_t r = cur / p.kt_total;  // split tile index
+    const int64_t tile_end = (r + 1) * p.kt_total;
     const int64_t e = end < tile_end ? end : tile_end;
-    it.tile = static_cast<int>(tile);
-    it.kt0 = static_cast<int>(cur - tile * p.kt_total);
+    it.tile = static_cast<int>(p.dp_tiles + r);
+    it.kt0 = static_cast<int>(cur - r * p.kt_total);
     it.kt1 = it.kt0 + static_cast<int>(e - cur);
-    it.slot = static_cast<int>(blockIdx.x - sk_owner(tile * p.kt_total, T, gridDim.x));
+    const SkOwners o = sk_tile_owners(r, p.kt_total, p.sk_unit, T, p.sk_grid);
+    it.slot = (o.first == o.last) ? -1 : static_cast<int>(blockIdx.x - o.first);
+    // The first owner reaches its part (the tile's first k steps) last of all
+    // its items, after the others have written theirs at the start of theirs.
+    it.nadd = (p.sk_inline && it.slot == 0) ? static_cast<int>(o.last - o.first) : 0;
     cur = e;
     return true;
   }
@@ -771,7 +787,9 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR, SPG>::kThreads, 1)
       float bias8[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) bias8[i] = 0.f;
-      if (it.slot < 0) {
+      const bool finisher = it.nadd > 0;
+      const bool writes_out = it.slot < 0 || finisher;
+      if (writes_out) {
         if constexpr (!GRP) {
           const ColConst cc = col_const<BF16, WK>(p, nn, col_ok);
           escale = (WK == kWFp8 || cc.fast) ? cc.s : 1.f;
@@ -786,9 +804,32 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR, SPG>::kThreads, 1)
           }
         }
       }
-      float* part = (it.slot >= 0)
-                        ? p.partial + (static_cast<int64_t>(it.tile) * p.max_slots + it.slot) * (BN * kWqNBlock)
-                        : nullptr;
+      const int64_t sk_r = static_cast<int64_t>(it.tile - p.dp_tiles);  // split tile index (stream-K items)
+      float* part = writes_out ? nullptr
+                               : p.partial + (sk_r * p.max_slots + it.slot) * (BN * kWqNBlock);
+      // Finisher: wait (bounded) until every other owner has written its partial
+      // of this tile; one thread polls, the barrier hands the result to all.
+      const float* others = nullptr;
+      if (finisher) {
+        bool ok = true;
+        if (et == 0) {
+          const uint64_t t0 = globaltimer();
+          for (int sl = 1; sl <= it.nadd && ok; ++sl) {
+            const uint64_t* flag = p.sk_flags + sk_r * p.max_slots + sl;
+            while (ld_acquire_gpu_u64(flag) != p.sk_token) {
+              if (*abort_flag || globaltimer() - t0 > WQMM_WAIT_NS) {
+                ok = false;
+                *abort_flag = 1;
+                atomicCAS(p.err, 0u, static_cast<uint32_t>(kDevTimeoutEpilogue));
+                break;
+              }
+            }
+          }
+        }
+        if (!named_bar_and(1, 128, ok)) break;
+        __threadfence();
+        others = p.partial + sk_r * p.max_slots * (BN * kWqNBlock);  // slot s at others + s * BN * 128
+      }
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += kER) {
         const bool last = (c0 + kER >= BN);
@@ -819,8 +860,22 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR, SPG>::kThreads, 1)
           for (int q = 0; q < kER; ++q) part[(c0 + q) * kWqNBlock + nl] = __uint_as_float(v[q]);
           continue;
         }
+        if (others) {
+          // the owners' partials in slot order after this CTA's own (slot 0)
+          float acc[kER];
 #pragma unroll
-        for (int q = 0; q < kER; ++q) stage[q * kWqNBlock + nl] = __uint_as_float(v[q]) * escale;
+          for (int q = 0; q < kER; ++q) acc[q] = __uint_as_float(v[q]);
+          for (int sl = 1; sl <= it.nadd; ++sl) {
+            const float* src = others + static_cast<int64_t>(sl) * (BN * kWqNBlock) + c0 * kWqNBlock + nl;
+#pragma unroll
+            for (int q = 0; q < kER; ++q) acc[q] += src[q * kWqNBlock];
+          }
+#pragma unroll
+          for (int q = 0; q < kER; ++q) stage[q * kWqNBlock + nl] = acc[q] * escale;
+        } else {
+#pragma unroll
+          for (int q = 0; q < kER; ++q) stage[q * kWqNBlock + nl] = __uint_as_float(v[q]) * escale;
+        }
         named_bar_sync(1, 128);
 #pragma unroll
         for (int ps = 0; ps < kPasses; ++ps) {
@@ -842,6 +897,12 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR, SPG>::kThreads, 1)
           }
         }
         named_bar_sync(1, 128);  // the staging tile is rewritten by the next chunk
+      }
+      if (part && p.sk_inline) {
+        // this owner's partial is complete: publish it to the tile's first owner
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (et == 0) st_release_gpu_u64(p.sk_flags + sk_r * p.max_slots + it.slot, p.sk_token);
       }
       ++j;
     }
@@ -1077,8 +1138,9 @@ constexpr int dgroups() {
 }
 
 // Turns of two k steps per dequantisation group (two groups) for wide m
-// tiles over whole tiles with an even number of k steps; one step per turn
-// (four groups) otherwise.
+// tiles with an even number of k steps, whose work items then all start on an
+// even step and have an even length (stream-K splits fall on pairs of steps);
+// one step per turn (four groups) otherwise.
 template <int BN, bool PAIR, int WK, bool BF16, int SPG>
 cudaError_t launch_spg(const CUtensorMap& tmap, const WqParams& p, int grid, cudaStream_t s) {
   constexpr int DG = SPG == 2 ? 2 : dgroups<BN>();
@@ -1093,7 +1155,8 @@ cudaError_t launch_spg(const CUtensorMap& tmap, const WqParams& p, int grid, cud
 template <int BN, bool PAIR, int WK, bool BF16>
 cudaError_t launch_mode(const CUtensorMap& tmap, const WqParams& p, int grid, cudaStream_t s) {
   if constexpr (BN >= 128 && !PAIR) {
-    if (!p.stream_k && p.kt_total % 2 == 0) return launch_spg<BN, PAIR, WK, BF16, 2>(tmap, p, grid, s);
+    if (p.kt_total % 2 == 0 && (!p.stream_k || p.sk_unit == 2))
+      return launch_spg<BN, PAIR, WK, BF16, 2>(tmap, p, grid, s);
   }
   return launch_spg<BN, PAIR, WK, BF16, 1>(tmap, p, grid, s);
 }
@@ -1109,38 +1172,88 @@ cudaError_t launch_bn(const CUtensorMap& tmap, const WqParams& p, int wk, bool b
 }
 
 // ---------------------------------------------------------------- stream-K fix-up
+// For every split tile with more than one owner:
 // out = (sum of the tile's partials, in slot order) * epilogue scale + bias + x3.
-// One 128-thread block row per (tile, m row); warp = 32 aligned columns, the
-// same grouping the GEMM's epilogue uses for its warp-uniform scale choice.
-__global__ void __launch_bounds__(128) wqmm_fixup_kernel(const FixupParams p) {
-  const int64_t rows = static_cast<int64_t>(p.num_tiles) * p.bn;
-  const int64_t T = static_cast<int64_t>(p.num_tiles) * p.kt_total;
-  const int nl = threadIdx.x;  // column within the 128-column block
+// A block takes 16 rows x 128 columns of one tile: thread = 8 consecutive
+// columns of one row, 16-byte loads of each partial, of bias and x3, one
+// 16-byte store.  The per-channel choice of applying the scale here is made per
+// 32 aligned columns (four threads), the grouping of the GEMM's dequantisation
+// warps.
+constexpr int kFixRows = 16;
+__global__ void __launch_bounds__(256) wqmm_fixup_kernel(const FixupParams p) {
+  const int64_t split = p.num_tiles - p.dp_tiles;  // tiles after the whole-tile waves
+  const int64_t T = split * p.kt_total / p.sk_unit;
+  const int rb_per_tile = p.bn / kFixRows;
+  const int64_t row_blocks = split * rb_per_tile;
+  const int c8 = (threadIdx.x & 15) * 8;  // this thread's first column within the 128-column block
+  const int rsub = threadIdx.x >> 4;      // its row within the block's 16
   const bool bf16 = p.act_bf16 != 0;
-  for (int64_t rr = blockIdx.x; rr < rows; rr += gridDim.x) {
-    const int tile = static_cast<int>(rr / p.bn);
-    const int ml = static_cast<int>(rr % p.bn);
+  for (int64_t rb = blockIdx.x; rb < row_blocks; rb += gridDim.x) {
+    const int64_t r = rb / rb_per_tile;  // split tile index (the same for the whole block)
+    const SkOwners o = sk_tile_owners(r, p.kt_total, p.sk_unit, T, p.sk_grid);
+    if (o.first == o.last) continue;     // one owner: the GEMM wrote this tile whole
+    const int tile = static_cast<int>(p.dp_tiles + r);
+    const int ml = static_cast<int>(rb % rb_per_tile) * kFixRows + rsub;
     const int nb = tile % p.num_nb;
     const int64_t mm = static_cast<int64_t>(tile / p.num_nb) * p.bn + ml;
-    const int nn = nb * kWqNBlock + nl;
-    const bool col_ok = nn < p.n;
-    const int64_t first = static_cast<int64_t>(tile) * p.kt_total;
-    const int slots = static_cast<int>(sk_owner(first + p.kt_total - 1, T, p.grid) - sk_owner(first, T, p.grid)) + 1;
-    float acc = 0.f;
-    for (int s = 0; s < slots; ++s)
-      acc += p.partial[((static_cast<int64_t>(tile) * p.max_slots + s) * p.bn + ml) * kWqNBlock + nl];
-    float escale = 1.f;
+    const int nn = nb * kWqNBlock + c8;
+    const bool col_ok = nn < p.n;  // n is a multiple of 32: 8 columns are all in or all out
+    const int slots = static_cast<int>(o.last - o.first) + 1;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    for (int sl = 0; sl < slots; ++sl) {
+      const float4* src =
+          reinterpret_cast<const float4*>(p.partial + ((r * p.max_slots + sl) * p.bn + ml) * kWqNBlock + c8);
+      const float4 a = src[0], b = src[1];
+      acc[0] += a.x, acc[1] += a.y, acc[2] += a.z, acc[3] += a.w;
+      acc[4] += b.x, acc[5] += b.y, acc[6] += b.z, acc[7] += b.w;
+    }
+    float escale[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) escale[e] = 1.f;
     if (p.mode != kPerGroup) {
-      const int idx = (p.mode == kPerTensor) ? 0 : (col_ok ? nn : 0);
-      const float off = p.offset ? act_f32(p.offset[idx], bf16) : 0.f;
-      const bool fast = __all_sync(kFull, small_int(off));
-      if (fast) escale = act_f32(p.scale[idx], bf16);
+      bool small = true;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int idx = (p.mode == kPerTensor) ? 0 : (col_ok ? nn + e : 0);
+        small = small && small_int(p.offset ? act_f32(p.offset[idx], bf16) : 0.f);
+      }
+      // the four threads of each 32-column group (lanes differing in bits 0-1) agree
+      small = small && __shfl_xor_sync(kFull, static_cast<int>(small), 1);
+      small = small && __shfl_xor_sync(kFull, static_cast<int>(small), 2);
+      if (small) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) escale[e] = act_f32(p.scale[(p.mode == kPerTensor) ? 0 : (col_ok ? nn + e : 0)], bf16);
+      }
     }
     if (col_ok && mm < p.m) {
-      float y = acc * escale;
-      if (p.bias) y += act_f32(p.bias[nn], bf16);
-      if (p.x3) y += act_f32(p.x3[mm * p.n + nn], bf16);
-      p.out[mm * p.n + nn] = f32_act(y, bf16);
+      float y[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[e] = acc[e] * escale[e];
+      if (p.bias) {
+        const uint4 bv = *reinterpret_cast<const uint4*>(p.bias + nn);
+        const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          y[2 * h] += act_f32(static_cast<uint16_t>(bw[h] & 0xFFFFu), bf16);
+          y[2 * h + 1] += act_f32(static_cast<uint16_t>(bw[h] >> 16), bf16);
+        }
+      }
+      if (p.x3) {
+        const uint4 xv = *reinterpret_cast<const uint4*>(p.x3 + mm * p.n + nn);
+        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          y[2 * h] += act_f32(static_cast<uint16_t>(xw[h] & 0xFFFFu), bf16);
+          y[2 * h + 1] += act_f32(static_cast<uint16_t>(xw[h] >> 16), bf16);
+        }
+      }
+      uint32_t ow[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h)
+        ow[h] = static_cast<uint32_t>(f32_act(y[2 * h], bf16)) | (static_cast<uint32_t>(f32_act(y[2 * h + 1], bf16)) << 16);
+      *reinterpret_cast<uint4*>(p.out + mm * p.n + nn) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
     }
   }
 }
@@ -1153,19 +1266,27 @@ int wqmm_ctas_per_sm(int bn, int wk) {
   return 1;  // every configuration uses most of the SM's shared memory for its ring
 }
 
+template <int BN>
+int pair_slots_bn(int wk, bool act_bf16) {
+  constexpr int DG = dgroups<BN>();
+  if (wk == kW4) return act_bf16 ? pair_slots_one<BN, DG, kW4, true>() : pair_slots_one<BN, DG, kW4, false>();
+  if (wk == kW8) return act_bf16 ? pair_slots_one<BN, DG, kW8, true>() : pair_slots_one<BN, DG, kW8, false>();
+  return act_bf16 ? pair_slots_one<BN, DG, kWFp8, true>() : pair_slots_one<BN, DG, kWFp8, false>();
+}
+
 int wqmm_pair_slots(int bn, int wk, bool act_bf16) {
-  if (bn != 192) return 0;  // CTA pairs are built for the 192-row m tile
-  constexpr int DG = dgroups<192>();
-  if (wk == kW4) return act_bf16 ? pair_slots_one<192, DG, kW4, true>() : pair_slots_one<192, DG, kW4, false>();
-  if (wk == kW8) return act_bf16 ? pair_slots_one<192, DG, kW8, true>() : pair_slots_one<192, DG, kW8, false>();
-  return act_bf16 ? pair_slots_one<192, DG, kWFp8, true>() : pair_slots_one<192, DG, kWFp8, false>();
+  // CTA pairs are built for the 192- and 256-row m tiles
+  if (bn == 192) return pair_slots_bn<192>(wk, act_bf16);
+  if (bn == 256) return pair_slots_bn<256>(wk, act_bf16);
+  return 0;
 }
 
 cudaError_t launch_wqmm_gemm(const CUtensorMap& tmap_x1, const WqParams& p, int bn, int wk, bool act_bf16,
                              int grid, cudaStream_t s) {
   if (p.pair) {
-    if (bn != 192) return cudaErrorInvalidValue;
-    return launch_bn<192, true>(tmap_x1, p, wk, act_bf16, grid, s);
+    if (bn == 192) return launch_bn<192, true>(tmap_x1, p, wk, act_bf16, grid, s);
+    if (bn == 256) return launch_bn<256, true>(tmap_x1, p, wk, act_bf16, grid, s);
+    return cudaErrorInvalidValue;
   }
   switch (bn) {
     case 16: return launch_bn<16, false>(tmap_x1, p, wk, act_bf16, grid, s);
@@ -1181,9 +1302,10 @@ cudaError_t launch_wqmm_gemm(const CUtensorMap& tmap_x1, const WqParams& p, int 
 cudaError_t launch_wqmm_fixup(const FixupParams& p, cudaStream_t s) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t rows = static_cast<int64_t>(p.num_tiles) * p.bn;
-  const int64_t cap = static_cast<int64_t>(sms) * 16;
-  wqmm_fixup_kernel<<<static_cast<unsigned>(rows < cap ? rows : cap), 128, 0, s>>>(p);
+  const int64_t blocks = static_cast<int64_t>(p.num_tiles - p.dp_tiles) * (p.bn / kFixRows);
+  if (blocks <= 0) return cudaSuccess;
+  const int64_t cap = static_cast<int64_t>(sms) * 8;  // 256-thread blocks: 8 per SM fill it
+  wqmm_fixup_kernel<<<static_cast<unsigned>(blocks < cap ? blocks : cap), 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 

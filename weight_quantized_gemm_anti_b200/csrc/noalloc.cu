@@ -69,8 +69,10 @@ extern "C" wqmm_status wqmm_matmul_no_alloc(const wqmm_tensor* x1, const wqmm_te
                                             const wqmm_tensor* output, wqmm_stream stream) {
   uint64_t need = 0;
   wqmm_executor* ex = nullptr;
+  wqmm::g_plan_ws_cap = kScratchBytes;  // plan within the fixed array where a plan can
   wqmm_status st = wqmm_get_workspace_size(x1, x2, bias, antiquant_scale, antiquant_offset, x3, group, reduce_op,
                                            comm_turn, stream_mode, antiquant_group_size, output, &need, &ex);
+  wqmm::g_plan_ws_cap = 0;
   if (st != WQMM_SUCCESS) return st;
   if (need > kScratchBytes) {
     wqmm_executor_destroy(ex);

@@ -226,6 +226,17 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// gpu-scope acquire load / release store of a 64-bit word in global memory
+// (flags between CTAs of one grid).
+__device__ __forceinline__ uint64_t ld_acquire_gpu_u64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu_u64(uint64_t* p, uint64_t v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
 // Named barrier `id` over `count` threads (whole warps), for roles that
 // synchronise among themselves only; id 0 is __syncthreads'.
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
