@@ -284,13 +284,6 @@ __device__ __forceinline__ void dq8_group_half(const uint4 chA, const uint4 chB,
   }
 }
 
-// Scale/offset bits of one column for the two 32-wide halves of a k step
-// (per-group mode).
-struct GroupSO {
-  uint16_t s[2], o[2];
-  bool one_row;  // warp-uniform: both halves use the same group row (and lie inside k)
-};
-
 // Group row of half index hidx = 2*kt (+1 for the second half): row = hidx / gq,
 // gq = G / 32 halves per group.  Advanced without division along a group's
 // k steps.
@@ -309,7 +302,6 @@ struct GroupRow {
       ++row;
     }
   }
-  __device__ __forceinline__ int row1(int gq) const { return row + (rem + 1 >= gq ? 1 : 0); }
 };
 
 // Position in a ring of N slots (and its phase parity) of the k steps one
@@ -332,21 +324,6 @@ struct Cursor {
     i = j;
   }
 };
-
-__device__ __forceinline__ GroupSO load_group_so(const WqParams& p, int kt, const GroupRow& gr, int gq, int nn,
-                                                 bool col_ok) {
-  GroupSO r;
-  const int rows[2] = {gr.row, gr.row1(gq)};
-  r.one_row = rows[0] == rows[1] && kt * kWqKTile + 32 < p.k;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const bool use = col_ok && (kt * kWqKTile + 32 * h < p.k);
-    const int64_t idx = static_cast<int64_t>(rows[h]) * p.n + nn;
-    r.s[h] = use ? __ldg(p.scale + idx) : uint16_t(0);
-    r.o[h] = (use && p.offset) ? __ldg(p.offset + idx) : uint16_t(0);
-  }
-  return r;
-}
 
 // Scale/offset bits of one column for the NH 32-wide halves of one turn of a
 // dequantisation group (NH = 2 SPG), per-group mode.
