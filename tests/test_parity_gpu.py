@@ -243,6 +243,35 @@ def test_wqmm_split_last_wave_parity(spec, monkeypatch):
     assert rel_err(g, whole) <= TOL[case.act]
 
 
+def test_wqmm_inline_stream_k_graph_replays(monkeypatch):
+    # A launch recorded into a CUDA graph replays with the same flag token: each
+    # replay must still wait for its own owners' partials (the first owner
+    # clears the flags it consumed).  x1 changes between replays, so partials
+    # left from an earlier replay would show in the result.
+    import dataclasses
+    monkeypatch.setenv("WQMM_GRID", "8")
+    monkeypatch.setenv("WQMM_PAIR", "0")
+    case = WL.make_wqmm_case(name="graph_sk", x1_shape=(40, 512), n=2304, act="bf16", wdt="i4", mode="group",
+                             group_size=64, scale_range=(0.005, 0.05), offset_range=(-4, 4), seed=7)
+    d = C.wqmm_to_device(case)
+    ws = C.wqmm_call(d)
+    torch.cuda.synchronize()
+    assert ws is not None and ws.numel() > 0
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        C.wqmm_call(d, workspace=ws)
+    for r in range(3):
+        x1 = WL.act_bits(np.random.default_rng(100 + r).standard_normal(size=case.x1_shape), case.act)
+        d.x1.view(torch.int16).copy_(torch.from_numpy(np.ascontiguousarray(x1).view(np.int16)).to(d.x1.device))
+        g.replay()
+        torch.cuda.synchronize()
+        no_device_error()
+        ye, _ = oracle.wqmm(dataclasses.replace(case, x1=x1))
+        got = dec(gpu_bits(d.out), case.act)
+        assert rel_err(got, ye) <= TOL[case.act], f"replay {r}: rel err {rel_err(got, ye):.3e}"
+    del g
+
+
 def test_wqmm_cta_pair_matches_single_cta(monkeypatch):
     # the same problem with and without CTA pairs: both within tolerance of the
     # oracle, and close to each other

@@ -802,6 +802,10 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR, SPG>::kThreads, 1)
               }
             }
           }
+          // This CTA is the flags' only reader: clear them, so that a replay of
+          // this launch (a CUDA graph reuses the token) waits for its own writes.
+          if (ok)
+            for (int sl = 1; sl <= it.nadd; ++sl) p.sk_flags[sk_r * p.max_slots + sl] = 0;
         }
         if (!named_bar_and(1, 128, ok)) break;
         __threadfence();
