@@ -222,7 +222,15 @@ WQMM_API wqmm_status wqmm_stream_wait(wqmm_stream stream, int32_t timeout_ms);
 
 /* Read the library's device error word: 0, or the code of the first bounded
  * in-kernel wait that gave up (the kernel then ended early and its output is
- * invalid).  Synchronous with respect to the device; `reset` != 0 clears it. */
+ * invalid).  Synchronous with respect to the device; `reset` != 0 clears it.
+ * Codes: 1 a copy producer, 2 the MMA issuer, 3 a dequantiser, 4 the epilogue
+ * (including the wait of a split tile's first owner for the other owners'
+ * partials), 5 the final drain of outstanding copies.
+ * After a timeout, owners that finished late may have left "partial written"
+ * flags set in the workspace.  A new wqmm_run call never matches them (each
+ * launch waits for a token of its own), but a CUDA graph replays a captured
+ * launch with its captured token: zero the graph's workspace before replaying
+ * it once a timeout has been reported. */
 WQMM_API wqmm_status wqmm_device_error(uint32_t* code, int32_t reset);
 
 /* Library version string, e.g. "wqmm 0.1 sm_100a". */

@@ -66,7 +66,7 @@ def lib():
             L.oracle_weight_at.argtypes = [I32, P, I64, I64, I64, I64]
             L.oracle_weight_at.restype = D
             L.oracle_wqmm.argtypes = [I64, I64, I64, I32, P, I32, P, I64, I64, I32, I64, P, P, I64, I64,
-                                      P, P, I64, P, I64, P, I32, P, P]
+                                      P, P, I64, P, I64, P, P, P]
             L.oracle_wqmm.restype = I32
             L.oracle_qmm.argtypes = [I64, I64, I64, P, P, I64, I64, P, I32, P, I64, P, I32, P,
                                      I64, P, I64, P, P, P, P]
@@ -113,8 +113,7 @@ def weight_at(wdt: str, x2: np.ndarray, s0: int, s1: int, kk: int, nn: int) -> f
 
 # ----------------------------------------------------------------- wqmm
 def wqmm_raw(*, m, k, n, act, x1, wdt, x2, x2_strides, mode, group_size, scale, offset, scale_strides,
-             bias=None, x3=None, rows: Optional[Sequence[int]] = None, cols: Optional[Sequence[int]] = None,
-             mirror=False):
+             bias=None, x3=None, rows: Optional[Sequence[int]] = None, cols: Optional[Sequence[int]] = None):
     """Evaluate the anti-quant GEMM on the selected rows x cols.
     Returns (y_exact float64 [R, C], y_rounded uint16 [R, C] in the activation format)."""
     x1 = np.ascontiguousarray(x1, dtype=np.uint16)
@@ -131,19 +130,18 @@ def wqmm_raw(*, m, k, n, act, x1, wdt, x2, x2_strides, mode, group_size, scale, 
     yr = np.empty((R, C), dtype=np.uint16)
     rc = lib().oracle_wqmm(m, k, n, _ACT[act], _p(x1), _WDT[wdt], _p(x2), int(x2_strides[0]), int(x2_strides[1]),
                            _MODE[mode], int(group_size), _p(scale), _p(offset), int(scale_strides[0]),
-                           int(scale_strides[1]), _p(bias), _p(x3), R, _p(r), C, _p(c), int(bool(mirror)),
-                           _p(ye), _p(yr))
+                           int(scale_strides[1]), _p(bias), _p(x3), R, _p(r), C, _p(c), _p(ye), _p(yr))
     if rc != 0:
         raise ValueError("oracle_wqmm rejected its arguments")
     return ye, yr
 
 
-def wqmm(case, rows=None, cols=None, mirror=False):
+def wqmm(case, rows=None, cols=None):
     """Oracle for a ``workloads.WqmmCase`` (output flattened to (m, n) / sampled)."""
     return wqmm_raw(m=case.m, k=case.k, n=case.n, act=case.act, x1=case.x1, wdt=case.wdt, x2=case.x2,
                     x2_strides=case.x2_strides, mode=case.mode, group_size=case.group_size, scale=case.scale,
                     offset=case.offset, scale_strides=case.scale_strides, bias=case.bias, x3=case.x3,
-                    rows=rows, cols=cols, mirror=mirror)
+                    rows=rows, cols=cols)
 
 
 # ----------------------------------------------------------------- qmm

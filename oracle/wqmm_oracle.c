@@ -190,16 +190,13 @@ static int check_selection(int64_t m, int64_t n, int64_t n_rows, const int64_t* 
  * scale/offset element (r, c) sits at r*ss0 + c*ss1 (per-tensor: index 0).
  *
  * rows/cols select which outputs to evaluate (NULL = all); outputs are written
- * densely as n_rows x n_cols.  mirror != 0 rounds every W[k][j] to the
- * activation format before the product (a diagnostic of what a
- * dequantise-then-MMA kernel sees; never used for grading).
- * Returns 0, or -1 on a bad argument.
+ * densely as n_rows x n_cols.  Returns 0, or -1 on a bad argument.
  */
 int oracle_wqmm(int64_t m, int64_t k, int64_t n, int act_dtype, const uint16_t* x1, int w_dtype,
                 const void* x2, int64_t s0, int64_t s1, int mode, int64_t group_size,
                 const uint16_t* scale, const uint16_t* offset, int64_t ss0, int64_t ss1,
                 const uint16_t* bias, const uint16_t* x3, int64_t n_rows, const int64_t* rows,
-                int64_t n_cols, const int64_t* cols, int mirror, double* y_exact, uint16_t* y_rounded) {
+                int64_t n_cols, const int64_t* cols, double* y_exact, uint16_t* y_rounded) {
     if (m < 0 || k < 0 || n < 0) return -1;
     if (act_dtype != OR_F16 && act_dtype != OR_BF16) return -1;
     if (w_dtype != OR_I8 && w_dtype != OR_I4 && w_dtype != OR_FP8E4M3) return -1;
@@ -222,9 +219,7 @@ int oracle_wqmm(int64_t m, int64_t k, int64_t n, int act_dtype, const uint16_t* 
                 int64_t sidx = (mode == OR_PER_TENSOR) ? 0 : r * ss0 + c * ss1;
                 double s = decode_act(act_dtype, scale[sidx]);
                 double o = offset ? decode_act(act_dtype, offset[sidx]) : 0.0;
-                double w = (oracle_weight_at(w_dtype, x2, s0, s1, kk, j) + o) * s;
-                if (mirror) w = decode_act(act_dtype, encode_act(act_dtype, w));
-                wcol[kk] = w;
+                wcol[kk] = (oracle_weight_at(w_dtype, x2, s0, s1, kk, j) + o) * s;
             }
             for (int64_t ii = 0; ii < n_rows; ++ii) {
                 int64_t i = rows ? rows[ii] : ii;

@@ -508,7 +508,15 @@ extern "C" wqmm_status wqmm_get_workspace_size(const wqmm_tensor* x1, const wqmm
         if (o.last - o.first + 1 > ms) ms = static_cast<int>(o.last - o.first + 1);
       }
       const uint64_t partial_bytes = static_cast<uint64_t>(split) * ms * ex->bn * kWqNBlock * 4;
-      if (!(dp > 0 && g_plan_ws_cap > 0 && partial_bytes > g_plan_ws_cap)) {
+      // A caller with a fixed workspace (g_plan_ws_cap) gets a schedule without
+      // split tiles when their partials and flags would not fit beside the
+      // other workspace regions: whole tiles are slower for these shapes but
+      // need no workspace of their own.
+      uint64_t other = 0;
+      if (!(x2->format == WQMM_FORMAT_PACKED)) other = round_up(packed_bytes_for(x2->dtype, k, n, false), 256);
+      if (mode == kPerGroup && scale_t) other += (offset ? 2 : 1) * round_up(static_cast<uint64_t>(ng) * n * 2, 256);
+      const uint64_t sk_bytes = round_up(partial_bytes, 256) + round_up(static_cast<uint64_t>(split) * ms * 8, 256);
+      if (!(g_plan_ws_cap > 0 && other + sk_bytes > g_plan_ws_cap)) {
         ex->stream_k = 1;
         ex->dp_tiles = static_cast<int>(dp);
         ex->sk_unit = unit;

@@ -6,8 +6,10 @@
 // the tcgen05 A operand held in tensor memory and x1 is the B operand in
 // shared memory.  A persistent, warp-specialised kernel, one CTA per SM:
 //
-//   warp 0      x1 producer: per 64-wide k step, the x1 tile (one 2-D tensor
-//               copy, 128-byte swizzle) into the x1 ring, which the MMA reads;
+//   warps 0 and 7 + 4 DG
+//               x1 producers, alternate k steps: per 64-wide k step, the x1
+//               tile (one 2-D tensor copy, 128-byte swizzle) into the x1 ring,
+//               which the MMA reads;
 //   warp 6      weight producer: the packed 128-column weight tile (one 1-D
 //               bulk copy) into the weight ring, which the dequantisers read
 //               and release as soon as the tile is in registers -- so weights
@@ -27,10 +29,16 @@
 //               in registers and tcgen05.st's them into one of its own TMEM A
 //               stages, so DG k steps are dequantised concurrently.
 //
-// Work is either whole output tiles dealt round-robin to the CTAs, or (few
-// tiles: small m) all k steps of all tiles split evenly over the CTAs
-// ("stream-K"); then every CTA writes fp32 partial tiles and a second kernel
-// sums them in a fixed order (deterministic, no inter-CTA waiting).
+// Work is whole output tiles dealt round-robin to the CTAs, optionally
+// followed by "stream-K" tiles whose k steps are split evenly over the CTAs
+// (few tiles, or the partly filled last wave of narrow tiles).  A split tile's
+// owners each produce an fp32 partial.  With at most four owners, the owner of
+// the tile's first k steps -- which reaches that part last of all its items --
+// waits (bounded, on per-launch-token flags) for the others' partials and adds
+// them in slot order in its own epilogue; with more owners, every owner writes
+// a partial and wqmm_fixup_kernel sums them.  Both orders are fixed, so
+// repeated runs agree bit for bit.  The inline wait assumes the persistent
+// CTAs of a launch are resident together (one per SM, grid <= SM count).
 //
 // Dequantisation, per element pair in bf16x2 / f16x2 registers:
 //   int4, integer offsets (warp-uniform test): t = 0x4300|nibble (= 128+q+8)

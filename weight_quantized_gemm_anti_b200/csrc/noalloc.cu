@@ -16,9 +16,12 @@
 //    rejected with WQMM_ERR_WORKSPACE before anything is launched;
 //  * all calls on a device share the one array, so calls whose work overlaps on
 //    the GPU (different streams, or other threads) race on it -- serialise them;
-//  * the array keeps whatever the previous call left in it; nothing needs
-//    clearing, because every byte a call reads from it was written earlier in
-//    that same call;
+//  * the array keeps whatever the previous call left in it.  Stale fp32
+//    partial tiles are never read: a tile's partials are read only after the
+//    owners of this launch have written them and raised their flags.  Stale
+//    "partial written" flags cannot match either: every launch waits for its
+//    own 64-bit token, which no earlier launch wrote, and the CTA that consumes
+//    a tile's flags clears them;
 //  * the first call on a device looks up the array's device address
 //    (cudaGetSymbolAddress, with that device current); make that first call
 //    before any stream capture begins.
