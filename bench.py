@@ -34,6 +34,8 @@ HEADLINE = "w4a16_g128_bf16_4096x4096x4096"
 METRIC = "anti-quant GEMM TFLOP/s & % of roofline (W4A16 g128, m=k=n=4096), 1 B200"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ["weight_quantized_gemm_anti_b200/csrc/kernels_wqmm.cu",
+                  "weight_quantized_gemm_anti_b200/csrc/kernels_smallm.cu",
+                  "weight_quantized_gemm_anti_b200/csrc/wqmm_common.cuh",
                   "weight_quantized_gemm_anti_b200/csrc/ptx.cuh",
                   "weight_quantized_gemm_anti_b200/csrc/kernels_qmm.cu",
                   "weight_quantized_gemm_anti_b200/csrc/kernels_aux.cu"]
@@ -80,8 +82,22 @@ def wqmm_schedule(m: int, n: int, k: int, sms: int) -> dict:
     num_nb = -(-n // 128)
     kt = -(-k // 64)
     tiles = -(-m // bn) * num_nb
-    out = {"bn": bn, "stream_k": False, "inline": False, "partial_bytes": 0, "flag_bytes": 0}
-    if k == 0 or kt < 2:
+    out = {"bn": bn, "stream_k": False, "inline": False, "partial_bytes": 0, "flag_bytes": 0,
+           "kernel": "smallm" if bn <= 32 else "general", "grid": min(tiles, sms)}
+    if k == 0:
+        return out
+    if bn <= 32:
+        # small-m kernel: stream-K over every tile, >= 16 k steps per CTA
+        unit = 2 if kt % 2 == 0 else 1
+        T = tiles * kt // unit
+        grid = max(1, min(sms, -(-(T * unit) // 16)))
+        owner = lambda s: ((s + 1) * grid - 1) // T
+        ms = max(owner((r * kt + kt - 1) // unit) - owner(r * kt // unit) + 1 for r in range(tiles))
+        out.update(stream_k=True, inline=ms <= 4, grid=grid)
+        if ms > 1:
+            out.update(partial_bytes=tiles * ms * bn * 128 * 4, flag_bytes=tiles * ms * 8 if ms <= 4 else 0)
+        return out
+    if kt < 2:
         return out
     rem = tiles % sms
     if tiles < sms:
@@ -98,7 +114,7 @@ def wqmm_schedule(m: int, n: int, k: int, sms: int) -> dict:
     owner = lambda s: ((s + 1) * skg - 1) // T
     ms = max(owner((r * kt + kt - 1) // unit) - owner(r * kt // unit) + 1 for r in range(split))
     out.update(stream_k=True, inline=ms <= 4, partial_bytes=split * ms * bn * 128 * 4,
-               flag_bytes=split * ms * 8 if ms <= 4 else 0)
+               flag_bytes=split * ms * 8 if ms <= 4 else 0, grid=grid)
     return out
 
 

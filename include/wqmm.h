@@ -241,6 +241,16 @@ WQMM_API const char* wqmm_version(void);
  * m * n int32 (row-major).  Call between phase 1 and phase 2. */
 WQMM_API wqmm_status qmm_debug_set_raw_accumulator(wqmm_executor* executor, void* acc_i32_out);
 
+/* Test-only: make the bounded device wait of a split tile's first owner (the
+ * wait for the other owners' fp32 partials of a stream-K plan) give up after
+ * `wait_ns` nanoseconds instead of 2 s (0 keeps 2 s), and, when `mismatch` is
+ * non-zero, wait for a flag value that no owner of the launch writes -- so the
+ * wait runs out, the kernel records error code 4 in the device error word
+ * (wqmm_device_error), ends early and leaves its output invalid.  No GPU fault
+ * is involved.  Call between phase 1 and phase 2 of wqmm; it has no effect on
+ * a plan without split tiles. */
+WQMM_API wqmm_status wqmm_debug_set_flag_wait(wqmm_executor* executor, uint64_t wait_ns, int32_t mismatch);
+
 #ifdef __cplusplus
 }
 #endif

@@ -117,6 +117,76 @@ def test_wqmm_small_parity(spec):
     check_wqmm(case)
 
 
+# ---------------------------------------------------------------- small m (m <= 32)
+# The small-m kernel: dequantisation groups that issue their own MMAs, x1
+# fetched per turn by the groups, per-group scale/offset rows staged with the
+# weights.  Even k-step counts take two-step turns, odd ones single steps; the
+# m tile is 16 rows (m <= 16) or 32.  k tails (k % 64 == 32) and ragged m and
+# n, every weight type and mode, and a tile split over many CTAs (fix-up).
+SMALLM = [
+    # name, x1_shape, n, act, wdt, mode, G, extras
+    ("sm_i4_g64_bf16_m16_odd_ksteps", (16, 320), 384, "bf16", "i4", "group", 64, {}),
+    ("sm_i4_g32_f16_m7", (7, 1024), 256, "f16", "i4", "group", 32, {}),
+    ("sm_i8_g64_bf16_m32_x3", (32, 768), 320, "bf16", "i8", "group", 64, {}),
+    ("sm_i8_chan_bf16_k_tail", (12, 96), 160, "bf16", "i8", "channel", 0, {}),
+    ("sm_i8_g32_f16_k_tail", (9, 160), 96, "f16", "i8", "group", 32, {}),
+    ("sm_fp8_chan_bf16_m30", (30, 640), 256, "bf16", "fp8", "channel", 0, {"offset": False}),
+    ("sm_i4_tensor_bf16_m3", (3, 2048), 512, "bf16", "i4", "tensor", 0, {}),
+    ("sm_i4_g128_bf16_fractional", (16, 512), 256, "bf16", "i4", "group", 128, {"fractional_offset": True}),
+    ("sm_i4_g64_bf16_m25_3d", (5, 5, 1024), 640, "bf16", "i4", "group", 64, {}),
+    ("sm_i4_g64_bf16_many_owners_fixup", (16, 8192), 128, "bf16", "i4", "group", 64, {}),
+    ("sm_i8_g96_bf16_rows_straddle", (20, 576), 128, "bf16", "i8", "group", 96, {}),
+]
+
+
+@pytest.mark.parametrize("spec", SMALLM, ids=[s[0] for s in SMALLM])
+def test_wqmm_small_m_kernel_parity(spec):
+    name, x1s, n, act, wdt, mode, G, extra = spec
+    case = WL.make_wqmm_case(name=name, x1_shape=x1s, n=n, act=act, wdt=wdt, mode=mode, group_size=G,
+                             seed=zlib.crc32(name.encode()) % 10000, **extra)
+    check_wqmm(case)
+
+
+@pytest.mark.parametrize("env", [{"WQMM_STREAMK": "0"}, {"WQMM_SMALLM": "0"}], ids=["whole_tiles", "general_kernel"])
+@pytest.mark.parametrize("spec", [SMALLM[0], SMALLM[2], SMALLM[5]], ids=[SMALLM[i][0] for i in (0, 2, 5)])
+def test_wqmm_small_m_other_schedules(spec, env, monkeypatch):
+    # the small-m kernel on whole tiles, and the general kernel's narrow m tiles
+    for key, val in env.items():
+        monkeypatch.setenv(key, val)
+    name, x1s, n, act, wdt, mode, G, extra = spec
+    case = WL.make_wqmm_case(name=name, x1_shape=x1s, n=n, act=act, wdt=wdt, mode=mode, group_size=G,
+                             seed=zlib.crc32(name.encode()) % 10000, **extra)
+    check_wqmm(case)
+
+
+def test_split_tile_flag_wait_runs_out_and_reports(monkeypatch):
+    # Failure detection without a GPU fault: the test hook makes the first
+    # owner of each split tile wait (bounded, 1 ms) for a flag value that no
+    # owner writes.  The kernel gives up, records code 4 (epilogue wait) in the
+    # device error word and returns; the next normal call is correct.
+    case = WL.make_wqmm_case(name="flag_timeout", x1_shape=(16, 2048), n=1024, act="bf16", wdt="i4", mode="group",
+                             group_size=64, scale_range=(0.005, 0.05), offset_range=(-4, 4), seed=41)
+    d = C.wqmm_to_device(case)
+    no_device_error()
+    D = W.desc
+    st, ws_size, ex = W.wqmm_get_workspace_size(D(d.x1), d.x2_desc, None if d.bias is None else D(d.bias),
+                                                d.scale_desc, d.offset_desc, None, None, "sum", 0, 1, d.group_size,
+                                                D(d.out))
+    assert st == W.SUCCESS and ws_size > 0  # split tiles: partials and flags in the workspace
+    ws = torch.zeros(ws_size, dtype=torch.uint8, device="cuda")
+    assert W.wqmm_debug_set_flag_wait(ex, 1_000_000, True) == W.SUCCESS
+    assert W.wqmm_run(ws.data_ptr(), ws_size, ex, None) == W.SUCCESS
+    assert W.wqmm_stream_wait(None, 10_000) == W.SUCCESS  # the kernel ended; nothing hung
+    st, code = W.wqmm_device_error(reset=True)
+    assert st == W.SUCCESS and code == 4
+    # the same problem, a fresh launch, the same workspace: correct again
+    C.wqmm_call(d, workspace=ws)
+    torch.cuda.synchronize()
+    no_device_error()
+    ye, _ = oracle.wqmm(case)
+    assert rel_err(dec(gpu_bits(d.out), "bf16"), ye) <= TOL["bf16"]
+
+
 # ---------------------------------------------------------------- CTA pairs
 # With the 192- or 256-row m tile (WQMM_BN), whole tiles per CTA (stream-K off)
 # and WQMM_PAIR=1, two CTAs of a cluster share each MMA (cta_group::2), each

@@ -84,9 +84,10 @@ def lib():
             L.wqmm_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), I32]
             L.wqmm_version.restype = ctypes.c_char_p
             L.qmm_debug_set_raw_accumulator.argtypes = [P, P]
+            L.wqmm_debug_set_flag_wait.argtypes = [P, ctypes.c_uint64, I32]
             for name in ("wqmm_get_workspace_size", "wqmm_run", "qmm_get_workspace_size", "qmm_run",
                          "wqmm_pack_weight_size", "wqmm_pack_weight", "wqmm_stream_wait", "wqmm_device_error",
-                         "qmm_debug_set_raw_accumulator"):
+                         "qmm_debug_set_raw_accumulator", "wqmm_debug_set_flag_wait"):
                 getattr(L, name).restype = I32
             _lib = L
     return _lib
@@ -215,6 +216,10 @@ def wqmm_version() -> str:
 
 def qmm_debug_set_raw_accumulator(executor, acc_ptr: int) -> int:
     return lib().qmm_debug_set_raw_accumulator(executor, acc_ptr)
+
+
+def wqmm_debug_set_flag_wait(executor, wait_ns: int, mismatch: bool) -> int:
+    return lib().wqmm_debug_set_flag_wait(executor, int(wait_ns), int(bool(mismatch)))
 
 
 def wqmm_matmul_no_alloc(x1, x2, bias, antiquant_scale, antiquant_offset, x3, group, reduce_op, comm_turn,

@@ -11,7 +11,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libwqmm.so")
-SOURCES = ["api.cu", "kernels_aux.cu", "kernels_wqmm.cu", "kernels_qmm.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "kernels_aux.cu", "kernels_wqmm.cu", "kernels_smallm.cu", "kernels_qmm.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I" + os.path.join(ROOT, "include")]

@@ -49,6 +49,7 @@ wqmm_status ok() {
   return WQMM_SUCCESS;
 }
 
+constexpr uint64_t kFlagWaitNs = 2000000000ull;  // a split tile's flag wait gives up after 2 s
 constexpr uint32_t kMagicLive = 0x57514D4Du;  // "WQMM"
 constexpr uint32_t kMagicDead = 0xDEADBEEFu;
 
@@ -92,6 +93,7 @@ struct wqmm_executor {
   int sk_grid = 0;     // stream-K: CTAs sharing the split tiles
   int sk_inline = 0;   // stream-K: the first owner of a split tile reduces it (no fix-up kernel)
   int pair = 0;        // 1: clusters of two CTAs share each MMA (256 weight columns per pair tile)
+  int smallm = 0;      // 1: the small-m kernel (m tile 16 or 32, DG MMA-issuing dequantisation groups)
   int num_pnb = 0;     // pair: 256-column blocks
   int num_tiles = 0;
   int max_slots = 0;
@@ -101,6 +103,10 @@ struct wqmm_executor {
   bool dq_per_tensor = false;
   const float* pertoken = nullptr;
   int32_t* raw_acc = nullptr;
+  // test hook (wqmm_debug_set_flag_wait): bound of a split tile's flag wait,
+  // and whether its first owner waits for a value no owner writes
+  uint64_t debug_wait_ns = 0;
+  bool debug_flag_mismatch = false;
 };
 
 namespace {
@@ -481,6 +487,42 @@ extern "C" wqmm_status wqmm_get_workspace_size(const wqmm_tensor* x1, const wqmm
     const char* sk_env = std::getenv("WQMM_STREAMK");
     const bool force_sk = sk_env && std::atoi(sk_env) == 1;
     const bool forbid_sk = sk_env && std::atoi(sk_env) == 0;
+    // m <= 32: the small-m kernel (WQMM_SMALLM=0 selects the general kernel).
+    // Its CTAs share the k steps of all tiles evenly (stream-K over every tile,
+    // at least 16 k steps per CTA, so that its four dequantisation groups each
+    // get several), unless WQMM_STREAMK=0 asks for whole tiles.
+    {
+      const char* sm_env = std::getenv("WQMM_SMALLM");
+      ex->smallm = (ex->bn == 16 || ex->bn == 32) && !(sm_env && std::atoi(sm_env) == 0) ? 1 : 0;
+    }
+    if (ex->smallm && !forbid_sk) {
+      // units of two k steps when the step count is even: the kernel then takes
+      // two-step turns, and every split point falls on a turn boundary
+      const int unit = kt % 2 == 0 ? 2 : 1;
+      const int64_t T = tiles * kt / unit;
+      int64_t grid = (T * unit + 15) / 16;
+      grid = grid < 1 ? 1 : (grid > slots ? slots : grid);
+      int ms = 1;
+      for (int64_t r = 0; r < tiles; ++r) {
+        const SkOwners o = sk_tile_owners(r, static_cast<int>(kt), unit, T, grid);
+        if (o.last - o.first + 1 > ms) ms = static_cast<int>(o.last - o.first + 1);
+      }
+      const uint64_t partial_bytes = ms > 1 ? static_cast<uint64_t>(tiles) * ms * ex->bn * kWqNBlock * 4 : 0;
+      uint64_t other = 0;
+      if (!(x2->format == WQMM_FORMAT_PACKED)) other = round_up(packed_bytes_for(x2->dtype, k, n, false), 256);
+      if (mode == kPerGroup && scale_t) other += (offset ? 2 : 1) * round_up(static_cast<uint64_t>(ng) * n * 2, 256);
+      const uint64_t sk_bytes = round_up(partial_bytes, 256) + round_up(static_cast<uint64_t>(tiles) * ms * 8, 256);
+      if (!(g_plan_ws_cap > 0 && ms > 1 && other + sk_bytes > g_plan_ws_cap)) {
+        ex->stream_k = 1;
+        ex->dp_tiles = 0;
+        ex->sk_unit = unit;
+        ex->sk_grid = static_cast<int>(grid);
+        ex->grid = static_cast<int>(grid);
+        ex->max_slots = ms;
+        ex->sk_inline = ms <= 4 ? 1 : 0;
+        if (const char* env = std::getenv("WQMM_SK_INLINE")) ex->sk_inline = (std::atoi(env) == 1 && ms <= 4) ? 1 : 0;
+      }
+    }
     // Stream-K: with fewer tiles than CTAs, the k steps of all tiles are spread
     // evenly over the CTAs.  With more, narrow m tiles (< 128 rows) run the whole
     // waves as whole tiles and split a last, partly filled wave (at most 85%
@@ -490,7 +532,7 @@ extern "C" wqmm_status wqmm_get_workspace_size(const wqmm_tensor* x1, const wqmm
     // dequantisers take two-step turns.
     const int64_t rem = tiles % slots;
     int64_t dp = -1;  // tiles run whole before the split ones; -1: no stream-K
-    if (!forbid_sk && kt >= 2) {
+    if (!ex->smallm && !forbid_sk && kt >= 2) {
       if (force_sk || tiles < slots)
         dp = 0;
       else if (ex->bn < 128 && rem > 0 && rem * 100 <= 85 * slots)
@@ -538,7 +580,7 @@ extern "C" wqmm_status wqmm_get_workspace_size(const wqmm_tensor* x1, const wqmm
     const char* pair_env = std::getenv("WQMM_PAIR");
     const int wk = x2->dtype == WQMM_DT_I4 ? kW4 : (x2->dtype == WQMM_DT_I8 ? kW8 : kWFp8);
     const bool want_pair = pair_env ? std::atoi(pair_env) == 1 : (ex->bn == 256 && wk == kW4);
-    if (!ex->stream_k && want_pair && (ex->bn == 192 || ex->bn == 256) && num_nb >= 2) {
+    if (!ex->smallm && !ex->stream_k && want_pair && (ex->bn == 192 || ex->bn == 256) && num_nb >= 2) {
       const int ps = pair_slots(ex->bn, wk, adt == WQMM_DT_BF16);
       if (ps > 0) {
         const int64_t pnb = (num_nb + 1) / 2;
@@ -561,7 +603,7 @@ extern "C" wqmm_status wqmm_get_workspace_size(const wqmm_tensor* x1, const wqmm
         ws = round_up(ws + ex->ws_offset.bytes, 256);
       }
     }
-    if (ex->stream_k) {
+    if (ex->stream_k && ex->max_slots > 1) {  // one owner per tile: no partials
       ex->ws_partial = {ws, static_cast<uint64_t>(tiles - ex->dp_tiles) * ex->max_slots * ex->bn * kWqNBlock * 4};
       ws = round_up(ws + ex->ws_partial.bytes, 256);
       if (ex->sk_inline) {
@@ -806,17 +848,21 @@ wqmm_status run_wqmm(void* ws, wqmm_executor* ex, cudaStream_t s) {
     }
   }
   CUtensorMap tmap;
-  wqmm_status st = make_tmap(&tmap, ex->x1, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                             2, ex->m, ex->k, kWqKTile, ex->pair ? ex->bn / 2 : ex->bn);
-  if (st) return st;
+  if (!ex->smallm) {  // the small-m kernel reads x1 with plain 16-byte copies
+    wqmm_status st = make_tmap(&tmap, ex->x1,
+                               bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ex->m,
+                               ex->k, kWqKTile, ex->pair ? ex->bn / 2 : ex->bn);
+    if (st) return st;
+  }
   WqParams p{};
+  p.x1 = static_cast<const uint16_t*>(ex->x1);
   p.wpack = wpack;
   p.scale = scale;
   p.offset = offset;
   p.bias = static_cast<const uint16_t*>(ex->bias);
   p.x3 = static_cast<const uint16_t*>(ex->x3);
   p.out = static_cast<uint16_t*>(ex->out);
-  p.partial = ex->stream_k ? reinterpret_cast<float*>(wsb + ex->ws_partial.offset) : nullptr;
+  p.partial = (ex->stream_k && ex->max_slots > 1) ? reinterpret_cast<float*>(wsb + ex->ws_partial.offset) : nullptr;
   p.err = device_error_word();
   p.m = ex->m;
   p.n = ex->n;
@@ -832,15 +878,18 @@ wqmm_status run_wqmm(void* ws, wqmm_executor* ex, cudaStream_t s) {
   p.sk_unit = ex->sk_unit;
   p.sk_grid = ex->sk_grid;
   p.sk_inline = ex->sk_inline;
-  p.sk_flags = ex->sk_inline ? reinterpret_cast<uint64_t*>(wsb + ex->ws_flags.offset) : nullptr;
+  p.sk_flags = (ex->sk_inline && ex->max_slots > 1) ? reinterpret_cast<uint64_t*>(wsb + ex->ws_flags.offset) : nullptr;
   p.sk_token = ex->sk_inline ? next_launch_token() : 0;
+  p.sk_expect = p.sk_token + (ex->debug_flag_mismatch ? 2 : 0);
+  p.sk_wait_ns = ex->debug_wait_ns > 0 ? ex->debug_wait_ns : kFlagWaitNs;
   p.max_slots = ex->max_slots;
   p.mode = ex->mode;
   p.group_size = ex->group_size;
   p.num_groups = ex->num_groups;
-  e = launch_wqmm_gemm(tmap, p, ex->bn, wk, bf16, ex->grid, s);
+  e = ex->smallm ? launch_wqmm_smallm(p, ex->bn, wk, bf16, ex->grid, s)
+                 : launch_wqmm_gemm(tmap, p, ex->bn, wk, bf16, ex->grid, s);
   if (e != cudaSuccess) return cuda_fail(e, "anti-quant GEMM launch");
-  if (ex->stream_k && !ex->sk_inline) {
+  if (ex->stream_k && !ex->sk_inline && ex->max_slots > 1) {
     FixupParams fp{};
     fp.partial = p.partial;
     fp.scale = scale;
@@ -1031,6 +1080,14 @@ extern "C" wqmm_status qmm_debug_set_raw_accumulator(wqmm_executor* executor, vo
   if (st) return st;
   if (acc_i32_out && !aligned16(acc_i32_out)) return fail(WQMM_ERR_PARAM_INVALID, "accumulator buffer must be 16-byte aligned");
   executor->raw_acc = static_cast<int32_t*>(acc_i32_out);
+  return ok();
+}
+
+extern "C" wqmm_status wqmm_debug_set_flag_wait(wqmm_executor* executor, uint64_t wait_ns, int32_t mismatch) {
+  wqmm_status st = take_executor(executor, OpKind::kWqmm);
+  if (st) return st;
+  executor->debug_wait_ns = wait_ns;
+  executor->debug_flag_mismatch = mismatch != 0;
   return ok();
 }
 

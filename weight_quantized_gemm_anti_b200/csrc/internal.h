@@ -26,6 +26,7 @@ constexpr int kQKTile = 128;
 constexpr int kQTileBytes = kQNBlock * kQKTile;
 
 struct WqParams {
+  const uint16_t* x1;     // (m, k) row-major activations (read directly by the small-m kernel)
   const uint8_t* wpack;   // packed weight (see above)
   const uint16_t* scale;  // raw f16/bf16 bits, (rows, n) row-major after any transpose
   const uint16_t* offset; // may be null
@@ -55,6 +56,9 @@ struct WqParams {
                           // kernel); 0 -- every owner writes a partial, the fix-up kernel reduces
   uint64_t* sk_flags;     // stream-K inline: [num_tiles - dp_tiles][max_slots] "partial written" flags
   uint64_t sk_token;      // stream-K inline: the value a flag holds once written in this launch
+  uint64_t sk_expect;     // stream-K inline: the value a tile's first owner waits for (sk_token;
+                          // another value only in the test hook that makes the wait run out)
+  uint64_t sk_wait_ns;    // stream-K inline: bound of that wait, in ns of %globaltimer
   int mode;               // QuantMode
   int group_size;         // per-group only
   int num_groups;         // rows of scale/offset in per-group mode
@@ -154,6 +158,9 @@ int wqmm_ctas_per_sm(int bn, int wk);
 int wqmm_pair_slots(int bn, int wk, bool act_bf16);
 cudaError_t launch_wqmm_gemm(const CUtensorMap& tmap_x1, const WqParams& p, int bn, int wk, bool act_bf16,
                              int grid, cudaStream_t s);
+// The small-m kernel (m tile of 16 or 32 rows, stream-K over all tiles); reads
+// x1 directly (p.x1), no tensor map.
+cudaError_t launch_wqmm_smallm(const WqParams& p, int bn, int wk, bool act_bf16, int grid, cudaStream_t s);
 cudaError_t launch_wqmm_fixup(const FixupParams& p, cudaStream_t s);
 cudaError_t launch_wqmm_epilogue(const EpiParams& p, cudaStream_t s);
 // tmap_w: the packed int8 weight viewed as rows of 128 bytes (box 128 x 128,

@@ -59,6 +59,13 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// Raise the transaction count of the current phase by `bytes` without an
+// arrival (several copies may be announced before the single arrival).
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
@@ -84,6 +91,39 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   while (true) {
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer() - t0 > WQMM_WAIT_NS) {
+      *abort = 1;
+      if (err_word) atomicCAS(err_word, 0u, code);
+      return false;
+    }
+  }
+}
+
+// try_wait with a suspend-time hint: the thread may be suspended in hardware
+// for up to `hint_ns` until the phase completes, instead of spinning.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait that sleeps in hardware: each try_wait may suspend the thread
+// for up to `hint_ns` (it wakes when the phase completes), so a waiting warp
+// issues a handful of instructions instead of a polling loop.  Gives up, as
+// mbar_wait does, on the abort flag or after WQMM_WAIT_NS.
+__device__ __forceinline__ bool mbar_wait_hint(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                               uint32_t* err_word, uint32_t code, uint32_t hint_ns = 200000u) {
+  if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
     if (*abort) return false;
     if (globaltimer() - t0 > WQMM_WAIT_NS) {
       *abort = 1;
@@ -158,6 +198,18 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// ------------------------------------------------------------------ shared-memory loads by address
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint16_t lds_u16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+
 // ------------------------------------------------------------------ async proxy fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -202,6 +254,13 @@ __device__ __forceinline__ void cp_async_16(void* dst, const void* src, uint32_t
                : "memory");
 }
 
+// Make `bar` track this thread's earlier cp.async copies: its pending count
+// rises by one now and falls by one when they have all landed, so the phase
+// cannot complete before them.
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // Close the calling thread's open cp.async group (empty if it issued none).
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 
@@ -213,6 +272,12 @@ __device__ __forceinline__ void cp_async_wait_group() {
 
 // Bring the 128-byte line holding p into L2.
 __device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
+// Bulk prefetch of `bytes` (a multiple of 16, src 16-byte aligned) into L2, no
+// shared memory and no completion to wait for.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 
 // Pair form of tma_load_2d (cta_group::2): the copy lands in this CTA's shared
 // memory and completes its bytes on an mbarrier given by its shared::cluster
@@ -241,6 +306,13 @@ __device__ __forceinline__ void st_release_gpu_u64(uint64_t* p, uint64_t v) {
 // synchronise among themselves only; id 0 is __syncthreads'.
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Arrive at named barrier `id` (expecting `count` threads in all) without
+// waiting: the threads that bar.sync on it wait for these arrivals.  Memory
+// accesses before the arrival are visible to those threads after their sync.
+__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // Named barrier that also returns the AND of `pred` over its threads, so that
