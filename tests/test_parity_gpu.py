@@ -148,7 +148,8 @@ def test_wqmm_small_m_kernel_parity(spec):
 
 
 @pytest.mark.parametrize("env", [{"WQMM_STREAMK": "0"}, {"WQMM_SMALLM": "0"}], ids=["whole_tiles", "general_kernel"])
-@pytest.mark.parametrize("spec", [SMALLM[0], SMALLM[2], SMALLM[5]], ids=[SMALLM[i][0] for i in (0, 2, 5)])
+@pytest.mark.parametrize("spec", [SMALLM[0], SMALLM[1], SMALLM[2], SMALLM[5], SMALLM[9]],
+                         ids=[SMALLM[i][0] for i in (0, 1, 2, 5, 9)])
 def test_wqmm_small_m_other_schedules(spec, env, monkeypatch):
     # the small-m kernel on whole tiles, and the general kernel's narrow m tiles
     for key, val in env.items():
