@@ -10,7 +10,10 @@ with the weight pre-packed (the packing is weight preparation, done once).
   e2e       : the same metric through the same C-ABI calls with HOST buffers:
               every step copies its inputs from pinned host memory and reads
               the output back, all inside the timed interval.
-  roofline  : the GEMM kernel against the measured dense bf16 peak.
+  roofline  : the GEMM kernel against its bound: the measured dense bf16 peak
+              (anti-quant and non-quantised GEMMs: bf16/f16 MMAs), the int8
+              peak measured in this run (the int8 GEMM), or the measured HBM
+              bandwidth, whichever roofline time is larger for the workload.
   cpu_baseline / --impl reference : the CPU oracle timed on a bounded sample.
 
 N > 1 (torchrun): N independent replicas (one problem per GPU, no collective on
@@ -73,20 +76,21 @@ def load_traffic(workload: str):
 
 
 # ------------------------------------------------------------------ schedule
-def wqmm_schedule(m: int, n: int, k: int, sms: int) -> dict:
+def wqmm_schedule(m: int, n: int, k: int, sms: int, nonquant: bool = False) -> dict:
     """The anti-quant GEMM's schedule as the library's phase 1 chooses it with
     no tuning overrides (a restatement of its planner, checked against the
     library's workspace sizes in the CPU tests): m tile, stream-K or whole
-    tiles, and whether a fix-up kernel follows the GEMM."""
+    tiles, and whether a fix-up kernel follows the GEMM.  ``nonquant``: a
+    16-bit weight of the x1 dtype, which always runs on the general kernel."""
     bn = 16 if m <= 16 else 32 if m <= 32 else 64 if m <= 64 else 128 if m <= 128 else 256
     num_nb = -(-n // 128)
     kt = -(-k // 64)
     tiles = -(-m // bn) * num_nb
     out = {"bn": bn, "stream_k": False, "inline": False, "partial_bytes": 0, "flag_bytes": 0,
-           "kernel": "smallm" if bn <= 32 else "general", "grid": min(tiles, sms)}
+           "kernel": "smallm" if bn <= 32 and not nonquant else "general", "grid": min(tiles, sms)}
     if k == 0:
         return out
-    if bn <= 32:
+    if bn <= 32 and not nonquant:
         # small-m kernel: stream-K over every tile, >= 16 k steps per CTA
         unit = 2 if kt % 2 == 0 else 1
         T = tiles * kt // unit
@@ -123,6 +127,7 @@ class ClockSampler:
     def __init__(self):
         self.proc = None
         self.path = None
+        self.skip = 0
 
     def start(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
@@ -135,6 +140,12 @@ class ClockSampler:
                                           "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return
+        # the timed region starts once the sampler is writing (at most 5 s)
+        t0 = time.time()
+        while time.time() - t0 < 5.0 and self.proc.poll() is None and os.path.getsize(self.path) == 0:
+            time.sleep(0.02)
+        self.skip = sum(1 for _ in open(self.path))  # samples taken before the timed region
 
     def stop(self, gpu_index: int):
         if self.proc is None:
@@ -144,10 +155,13 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        sm, mx, reasons = [], 0.0, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
-            for line in f:
+            lines = f.readlines()
+
+        def parse(rows):
+            sm, mx, reasons = [], 0.0, set()
+            for line in rows:
                 parts = [p.strip() for p in line.split(",")]
                 if len(parts) < 9 or not parts[0].isdigit() or int(parts[0]) != gpu_index:
                     continue
@@ -159,11 +173,118 @@ class ClockSampler:
                 for nm, v in zip(names, parts[5:9]):
                     if v.lower() == "active":
                         reasons.add(nm)
+            return sm, mx, reasons
+
+        # samples taken during the timed region; a region shorter than the
+        # sampling interval falls back to the samples taken just before it
+        sm, mx, reasons = parse(lines[self.skip:])
+        if not sm:
+            sm, mx, reasons = parse(lines)
         os.unlink(self.path)
         if not sm:
             return None
         sm.sort()
         return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workload labels
+def describe_weight(case) -> str:
+    """Human-readable weight/quantisation label of a workload."""
+    if not hasattr(case, "wdt"):
+        dq = "per-tensor" if case.dequant_scale.size == 1 else "per-channel"
+        pt = " + per-token scale" if case.pertoken_scale is not None else ""
+        return f"int8 x int8, {dq} {case.dq_dtype} dequantScale{pt}"
+    if case.mode == "none":
+        return f"{case.wdt} (non-quantised), no antiquant"
+    w = {"i4": "int4", "i8": "int8", "fp8": "fp8-e4m3"}[case.wdt]
+    mode = {"tensor": "per-tensor", "channel": "per-channel", "group": f"per-group g={case.group_size}"}[case.mode]
+    off = " + offset" if case.offset is not None else ""
+    return f"{w} packed, {mode} scale{off}"
+
+
+def arithmetic_dtype(case) -> str:
+    """The type the MMAs compute in: the activation type, or int8."""
+    return "i8" if not hasattr(case, "wdt") else case.act
+
+
+def roofline_bound(flops: float, nbytes: float, tensor_peak_tflops: float, hbm_gbs: float) -> str:
+    """'tensor' when the tensor-core time of the FLOPs exceeds the HBM time of
+    the algorithmic bytes, else 'hbm'."""
+    return "tensor" if flops / (tensor_peak_tflops * 1e12) >= nbytes / (hbm_gbs * 1e9) else "hbm"
+
+
+def measure_int8_peak(device: str, iters: int = 20):
+    """Dense int8 tensor throughput measured on this GPU: torch._int_mm (the
+    vendor library) and this library's int8 GEMM, both on an 8192^3 problem
+    (per-tensor dequantScale, no bias, x3 or per-token scale).  Returns the
+    larger, with both figures."""
+    import torch
+    import workloads as WL
+    import weight_quantized_gemm_anti_b200 as W
+    from weight_quantized_gemm_anti_b200 import cases as C
+
+    s = 8192
+    flops = 2.0 * s * s * s
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(iters):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / iters
+
+    out = {"shape": f"{s}x{s}x{s}", "iters": iters}
+    a = torch.randint(-127, 128, (s, s), dtype=torch.int8, device=device)
+    bt = torch.randint(-127, 128, (s, s), dtype=torch.int8, device=device)
+    try:
+        ms = timed(lambda: torch._int_mm(a, bt))
+        out["torch_int_mm_tops"] = round(flops / (ms * 1e-3) / 1e12, 1)
+    except RuntimeError as e:  # no int8 library GEMM for this device / build
+        out["torch_int_mm_tops"] = None
+        out["torch_int_mm_error"] = str(e).splitlines()[0][:120]
+    del a, bt
+    case = WL.make_qmm_case(name="int8_peak", x1_shape=(s, s), n=s, out="bf16", bias=False, x3=False,
+                            pertoken=False, dq_per_tensor=True, seed=99)
+    d = C.qmm_to_device(case, device=device)
+    D = W.desc
+    descs = (D(d.x1), d.x2_desc, None, None, d.dq_desc, None, None, "sum", 0, 1, D(d.out))
+    st, ws, ex = W.qmm_get_workspace_size(*descs)
+    W.check(st)
+    W.wqmm_executor_destroy(ex)
+    wsb = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
+
+    def own():
+        st, ws2, ex2 = W.qmm_get_workspace_size(*descs)
+        W.check(st)
+        W.check(W.qmm_run(wsb.data_ptr(), ws2, ex2, stream))
+
+    ms = timed(own)
+    out["qmm_tops"] = round(flops / (ms * 1e-3) / 1e12, 1)
+    del d, wsb
+    torch.cuda.empty_cache()
+    cands = [v for v in (out["torch_int_mm_tops"], out["qmm_tops"]) if v]
+    out["peak_tops"] = max(cands)
+    out["peak_from"] = "torch._int_mm" if out["peak_tops"] == out["torch_int_mm_tops"] else "this library's int8 GEMM"
+    return out
+
+
+def workload_roofline(prob, peaks, int8_peak):
+    """(bound, peak, unit, peak_source) of a workload's roofline."""
+    if prob.int8:
+        tpeak = int8_peak["peak_tops"] if int8_peak else 2.0 * peaks["bf16_tflops"]
+        tsrc = (f"int8 measured in this run ({int8_peak['peak_from']}, {int8_peak['shape']})" if int8_peak
+                else "2 x measured bf16 burst (nominal ratio)")
+    else:
+        tpeak, tsrc = peaks["bf16_tflops"], "bf16 burst"
+    bound = roofline_bound(prob.flops, prob.bytes, tpeak, peaks["hbm_gbs"])
+    if bound == "tensor":
+        return bound, tpeak, "TFLOP/s", tsrc
+    return bound, peaks["hbm_gbs"], "GB/s", "HBM copy"
 
 
 # ------------------------------------------------------------------ GPU arm
@@ -211,9 +332,9 @@ class Problem:
             b += c.dequant_scale.nbytes + (0 if c.pertoken_scale is None else 4 * c.m)
             b += 0 if c.x3 is None else 2 * c.m * c.n
             return b
-        wbytes = {"i4": 0.5, "i8": 1.0, "fp8": 1.0}[c.wdt]
+        wbytes = {"i4": 0.5, "i8": 1.0, "fp8": 1.0, "f16": 2.0, "bf16": 2.0}[c.wdt]
         b = c.m * c.k * 2 + c.k * c.n * wbytes + c.m * c.n * 2
-        b += c.scale.nbytes + (0 if c.offset is None else c.offset.nbytes)
+        b += (0 if c.scale is None else c.scale.nbytes) + (0 if c.offset is None else c.offset.nbytes)
         b += 0 if c.bias is None else 2 * c.n
         b += 0 if c.x3 is None else 2 * c.m * c.n
         return b
@@ -236,7 +357,8 @@ class Problem:
         m = 1
         for d in c.x1_shape[:-1]:
             m *= d
-        sched = wqmm_schedule(m, c.n, k, self.torch.cuda.get_device_properties(0).multi_processor_count)
+        sched = wqmm_schedule(m, c.n, k, self.torch.cuda.get_device_properties(0).multi_processor_count,
+                              nonquant=c.mode == "none")
         # the GEMM, plus the fix-up kernel when split tiles are reduced by one
         return 1 + (1 if sched["stream_k"] and not sched["inline"] else 0)
 
@@ -380,53 +502,59 @@ def gpu_arm(args):
     e2e_ms = max_over_ranks([e2e_ms], "cuda")[0]
 
     extra = {}
+    int8_peak = None
     if rank == 0 and world == 1 and not args.no_extra:
         import workloads as WL
+        int8_peak = measure_int8_peak(f"cuda:{local}")
         for nm in WL.WORKLOAD_NAMES:
             if nm == args.config:
                 continue
             p2 = Problem(nm, f"cuda:{local}")
-            tt, _ = time_device(p2, args.extra_steps, 3, flush_bytes)
-            ms = sum(tt) / len(tt)
-            bound_tensor = not (p2.case.m <= 64)
-            ent = {"ms_per_step": ms, "tflops": p2.flops / (ms * 1e-3) / 1e12,
-                   "gbs": p2.bytes / (ms * 1e-3) / 1e9}
-            if bound_tensor:
-                peak = peaks["bf16_tflops"] * (2.0 if p2.int8 else 1.0)
-                ent["roofline"] = {"bound": "tensor", "peak": peak, "unit": "TFLOP/s",
-                                   "frac": ent["tflops"] / peak,
-                                   "note": "int8 peak = 2 x measured bf16 (nominal ratio)" if p2.int8 else ""}
-            else:
-                ent["roofline"] = {"bound": "hbm", "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                   "frac": ent["gbs"] / peaks["hbm_gbs"]}
+            tt, _ = time_device(p2, max(args.extra_steps, 50), 3, flush_bytes)
+            tt.sort()
+            ms = tt[len(tt) // 2]  # median step
+            bound, peak, unit, src = workload_roofline(p2, peaks, int8_peak)
+            ent = {"ms_per_step": round(ms, 5), "stat": f"median of {len(tt)} steps",
+                   "weight": describe_weight(p2.case), "dtype": arithmetic_dtype(p2.case),
+                   "tflops": round(p2.flops / (ms * 1e-3) / 1e12, 2),
+                   "gbs": round(p2.bytes / (ms * 1e-3) / 1e9, 1), "launches_per_step": p2.launches_per_step()}
+            ach = ent["tflops"] if bound == "tensor" else ent["gbs"]
+            ent["roofline"] = {"bound": bound, "achieved": ach, "peak": peak, "unit": unit,
+                               "frac": round(ach / peak, 4), "peak_source": src}
             extra[nm] = ent
             del p2
             torch.cuda.empty_cache()
 
+    if rank == 0 and prob.int8 and int8_peak is None:
+        int8_peak = measure_int8_peak(f"cuda:{local}")
     if rank == 0:
         ms_step = max_ms / args.steps
         value = replica_throughput(prob.flops, world, args.steps, max_ms)
-        achieved = prob.flops / (ms_step * 1e-3) / 1e12
-        peak = peaks["bf16_tflops"]
+        bound, peak, unit, src = workload_roofline(prob, peaks, int8_peak)
+        achieved = (prob.flops / (ms_step * 1e-3) / 1e12 if bound == "tensor"
+                    else prob.bytes / (ms_step * 1e-3) / 1e9)
         traffic = load_traffic(args.config)
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; shapes/distributions of the workload)",
+            "vs_baseline": None, "dtype": arithmetic_dtype(prob.case),
+            "data": "synthetic (seeded; shapes/distributions of the workload)",
             "config": {"workload": args.config, "m": prob.case.m, "k": prob.case.k, "n": prob.case.n,
-                       "weight": "int4 packed, per-group g=128 scale+offset", "l2": "flushed before every step "
+                       "weight": describe_weight(prob.case), "l2": "flushed before every step "
                        "(512 MB write outside the timed interval)", "parallelism": f"replicas x{world}"},
             "e2e": {"value": round(replica_throughput(prob.flops, world, 1, e2e_ms), 3), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": prob.launches_per_step() * args.steps,
-            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+            "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
                          "frac": round(achieved / peak, 4), "traffic": traffic,
-                         "peak_source": f"{peak_src} bf16 burst"},
+                         "peak_source": f"{peak_src} {src}" if "measured in this run" not in src else src},
             "clocks": clocks,
             "host_phase1_us": round(host_p1 * 1e6, 1),
         }
         if extra:
             line["configs_measured"] = extra
+        if int8_peak:
+            line["int8_peak_measured"] = int8_peak
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(args.config, args.cpu_rows)
         print(json.dumps(line), flush=True)
@@ -477,7 +605,7 @@ def main():
     ap.add_argument("--impl", default="wqmm", choices=["wqmm", "reference"])
     ap.add_argument("--config", default=HEADLINE)
     ap.add_argument("--extra-steps", type=int, default=100)
-    ap.add_argument("--no-extra", action="store_true", help="skip the other four workloads")
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads and the int8 peak leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=1024)
     ap.add_argument("--ref-rows", type=int, default=8)

@@ -99,9 +99,14 @@ typedef struct CUstream_st* wqmm_stream; /* a cudaStream_t; NULL = the legacy de
  *  x1                (m, k) or (b, s, k), f16 or bf16, row-major contiguous (not transposed).
  *  x2                (k, n) weight: int8, int4 or fp8-e4m3; ND row-major, ND "transposed"
  *                    (strides (1, k): the last two axes swapped, stored (n, k)), or
- *                    WQMM_FORMAT_PACKED from wqmm_pack_weight.
+ *                    WQMM_FORMAT_PACKED from wqmm_pack_weight.  An x2 of the x1 dtype
+ *                    (f16 / bf16) selects the non-quantised scenario of the same
+ *                    operator family ("非量化场景" of npu_mm_all_reduce_base, "x2":
+ *                    its dtype then equals x1's): output = x1 @ x2 + bias + x3, with
+ *                    antiquant_scale and antiquant_offset NULL and G = 0.
  *  bias              optional, (n), dtype of x1.
- *  antiquant_scale   required, dtype of x1: per-tensor (1); per-channel (n) or (1, n);
+ *  antiquant_scale   required for int8 / int4 / fp8 weights (NULL otherwise:
+ *                    WQMM_ERR_PARAM_NULLPTR), dtype of x1: per-tensor (1); per-channel (n) or (1, n);
  *                    per-group (ceil(k / G), n) -- contiguous, or transposed (strides
  *                    (1, ceil(k/G))) exactly when x2 is transposed ("约束说明").
  *  antiquant_offset  optional, same shape, dtype and strides as the scale; ADDED to the
@@ -120,7 +125,7 @@ typedef struct CUstream_st* wqmm_stream; /* a cudaStream_t; NULL = the legacy de
  * Shape rules ("形状与范围约束"): 1 <= m <= 2^31-1, 0 <= k <= 65535, 1 <= n <= 65535;
  * m == 0 or n == 0 is rejected; k == 0 is accepted and yields bias + x3 (or zeros).
  * Alignment (the int8/int4 rule of the "产品相关的格式与对齐约束" section, adopted
- * for this device): int8 / fp8 weights need k % 32 == 0 and n % 32 == 0,
+ * for this device): int8 / fp8 / f16 / bf16 weights need k % 32 == 0 and n % 32 == 0,
  * int4 weights k % 64 == 0 and n % 64 == 0.  All data pointers must be 16-byte aligned.
  */
 WQMM_API wqmm_status wqmm_get_workspace_size(const wqmm_tensor* x1, const wqmm_tensor* x2, const wqmm_tensor* bias,
@@ -169,7 +174,8 @@ WQMM_API wqmm_status qmm_run(void* workspace, uint64_t workspace_size, wqmm_exec
  *
  * The B200 counterpart of aclnnCalculateMatmulWeightSizeV2 + aclnnTransMatmulWeight
  * (the weight-format conversion in the QuantMatmulAllReduceV2 sample): re-lays a
- * (k, n) weight (ND or ND-transposed; int8, int4 or fp8-e4m3) into the K-major
+ * (k, n) weight (ND or ND-transposed; int8, int4 or fp8-e4m3, or f16 / bf16 for
+ * the non-quantised scenario) into the K-major
  * tiles the GEMM kernels stream (128 n-rows x 64 k per tile for wqmm, 256 x 128
  * for qmm).  The packed weight is then passed with format WQMM_FORMAT_PACKED and
  * the same logical shape (k, n); packing is done once, outside the timed path.

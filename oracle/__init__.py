@@ -32,8 +32,8 @@ _lib = None
 
 F16, BF16, F32, I8, I4, FP8E4M3 = 1, 2, 3, 4, 5, 7
 _ACT = {"f16": F16, "bf16": BF16}
-_WDT = {"i8": I8, "i4": I4, "fp8": FP8E4M3}
-_MODE = {"tensor": 0, "channel": 1, "group": 2}
+_WDT = {"i8": I8, "i4": I4, "fp8": FP8E4M3, "f16": F16, "bf16": BF16}  # f16/bf16: non-quantised
+_MODE = {"tensor": 0, "channel": 1, "group": 2, "none": 0}
 
 
 def build(force: bool = False) -> str:
@@ -118,7 +118,7 @@ def wqmm_raw(*, m, k, n, act, x1, wdt, x2, x2_strides, mode, group_size, scale, 
     Returns (y_exact float64 [R, C], y_rounded uint16 [R, C] in the activation format)."""
     x1 = np.ascontiguousarray(x1, dtype=np.uint16)
     x2 = np.ascontiguousarray(x2)
-    scale = np.ascontiguousarray(scale, dtype=np.uint16)
+    scale = None if scale is None else np.ascontiguousarray(scale, dtype=np.uint16)
     offset = None if offset is None else np.ascontiguousarray(offset, dtype=np.uint16)
     bias = None if bias is None else np.ascontiguousarray(bias, dtype=np.uint16)
     x3 = None if x3 is None else np.ascontiguousarray(x3, dtype=np.uint16)

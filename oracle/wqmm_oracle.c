@@ -8,7 +8,11 @@
  *
  *  wqmm  -- aclnnWeightQuantMatmulAllReduce, "计算公式":
  *           output = x1 @ ((x2 + antiquantOffset) * antiquantScale) + bias + x3
- *           (the AllReduce is the identity for one rank).  The offset is ADDED
+ *           (the AllReduce is the identity for one rank).  The non-quantised
+ *           scenario of the same family (npu_mm_all_reduce_base, "x2": in the
+ *           "非量化场景" x2 has the dtype of x1; the repository README's
+ *           "非量化融合场景") has no antiquant factors: W = x2 as stored, which is
+ *           what a NULL scale selects here.  The offset is ADDED
  *           to the weight before the scale is applied.  Per-tensor scale has
  *           shape (1), per-channel (n) or (1,n), per-group (ceil(k/G), n) with
  *           row k//G used for weight row k ("约束说明", and the golden script
@@ -158,9 +162,10 @@ static uint16_t encode_act(int dt, double v) {
 /* Value of weight element (kk, nn) of x2, viewed as a (k, n) matrix whose
  * element (kk, nn) sits at logical linear index kk*s0 + nn*s1.
  * int4: two's-complement nibbles, two per byte, the even linear index in the
- * low nibble ("low nibble first"). */
+ * low nibble ("low nibble first").  f16 / bf16 (non-quantised): 16-bit codes. */
 double oracle_weight_at(int w_dtype, const void* x2, int64_t s0, int64_t s1, int64_t kk, int64_t nn) {
     int64_t idx = kk * s0 + nn * s1;
+    if (w_dtype == OR_F16 || w_dtype == OR_BF16) return decode_act(w_dtype, ((const uint16_t*)x2)[idx]);
     if (w_dtype == OR_I8) return (double)((const int8_t*)x2)[idx];
     if (w_dtype == OR_FP8E4M3) return oracle_e4m3_to_double(((const uint8_t*)x2)[idx]);
     /* OR_I4 */
@@ -188,6 +193,8 @@ static int check_selection(int64_t m, int64_t n, int64_t n_rows, const int64_t* 
  * W[k][j] = (x2[k][j] + off[r(k)][c(j)]) * scale[r(k)][c(j)],
  * r(k) = k / group_size in per-group mode, else 0; c(j) = j unless per-tensor.
  * scale/offset element (r, c) sits at r*ss0 + c*ss1 (per-tensor: index 0).
+ * scale == NULL: the non-quantised scenario, W[k][j] = x2[k][j]; x2 must then
+ * have the activation dtype and offset must be NULL.
  *
  * rows/cols select which outputs to evaluate (NULL = all); outputs are written
  * densely as n_rows x n_cols.  Returns 0, or -1 on a bad argument.
@@ -199,8 +206,12 @@ int oracle_wqmm(int64_t m, int64_t k, int64_t n, int act_dtype, const uint16_t* 
                 int64_t n_cols, const int64_t* cols, double* y_exact, uint16_t* y_rounded) {
     if (m < 0 || k < 0 || n < 0) return -1;
     if (act_dtype != OR_F16 && act_dtype != OR_BF16) return -1;
-    if (w_dtype != OR_I8 && w_dtype != OR_I4 && w_dtype != OR_FP8E4M3) return -1;
-    if (mode == OR_PER_GROUP && group_size <= 0) return -1;
+    if (scale == NULL) {
+        if (w_dtype != act_dtype || offset != NULL) return -1;
+    } else if (w_dtype != OR_I8 && w_dtype != OR_I4 && w_dtype != OR_FP8E4M3) {
+        return -1;
+    }
+    if (scale != NULL && mode == OR_PER_GROUP && group_size <= 0) return -1;
     if (rows == NULL) n_rows = m;
     if (cols == NULL) n_cols = n;
     if (check_selection(m, n, n_rows, rows, n_cols, cols)) return -1;
@@ -214,6 +225,10 @@ int oracle_wqmm(int64_t m, int64_t k, int64_t n, int act_dtype, const uint16_t* 
             int64_t j = cols ? cols[jj] : jj;
             /* decode weight column j: W[kk][j] */
             for (int64_t kk = 0; kk < k; ++kk) {
+                if (scale == NULL) {
+                    wcol[kk] = oracle_weight_at(w_dtype, x2, s0, s1, kk, j);
+                    continue;
+                }
                 int64_t r = (mode == OR_PER_GROUP) ? kk / group_size : 0;
                 int64_t c = (mode == OR_PER_TENSOR) ? 0 : j;
                 int64_t sidx = (mode == OR_PER_TENSOR) ? 0 : r * ss0 + c * ss1;

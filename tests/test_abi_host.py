@@ -27,7 +27,7 @@ def wq(x1=((32, 64), W.DT_F16), x2=((64, 128), W.DT_I8), scale=((128,), None), o
     adt = x1[1]
     x1d = T(x1[0], adt, data=FAKE if 0 not in x1[0] else 0)
     x2d = T(x2[0], x2[1], strides=x2_strides, data=FAKE if 0 not in x2[0] else 0, fmt=x2_fmt)
-    sd = T(scale[0], scale[1] or adt, strides=scale_strides)
+    sd = None if scale is None else T(scale[0], scale[1] or adt, strides=scale_strides)
     od = None if offset is None else T(offset[0], offset[1] or adt, strides=scale_strides)
     bd = None if bias is None else T(bias[0], bias[1] or adt)
     x3d = None if x3 is None else T(x3[0], x3[1] or adt)
@@ -93,7 +93,7 @@ def test_null_required_inputs():
 
 def test_dtype_rules():
     assert wq(x1=((32, 64), W.DT_I8))[0] == W.ERR_PARAM_INVALID                    # x1 not f16/bf16
-    assert wq(x2=((64, 128), W.DT_F16))[0] == W.ERR_PARAM_INVALID                  # non-quant weight
+    assert wq(x2=((64, 128), W.DT_F16))[0] == W.ERR_PARAM_INVALID                  # non-quant weight + scale
     assert wq(scale=((128,), W.DT_BF16))[0] == W.ERR_PARAM_INVALID                 # scale dtype != x1
     assert wq(offset=((128,), W.DT_BF16))[0] == W.ERR_PARAM_INVALID
     assert wq(bias=((128,), W.DT_F32))[0] == W.ERR_PARAM_INVALID
@@ -101,6 +101,25 @@ def test_dtype_rules():
     assert wq(out=((32, 128), W.DT_BF16))[0] == W.ERR_PARAM_INVALID
     assert wq(x1=((32, 64), W.DT_BF16), x2=((64, 128), W.DT_I4))[0] == W.SUCCESS
     assert wq(x2=((64, 128), W.DT_FP8E4M3))[0] == W.SUCCESS                         # per-channel fp8
+
+
+def test_non_quantised_rules():
+    # x2 of the x1 dtype: the non-quantised scenario, no antiquant factors
+    st, ws = wq(x2=((64, 128), W.DT_F16), scale=None)
+    assert st == W.SUCCESS and ws >= 64 * 128 * 2                                # the 16-bit weight re-laid
+    assert wq(x1=((32, 64), W.DT_BF16), x2=((64, 128), W.DT_BF16), scale=None, bias=((128,), None),
+              x3=((32, 128), None))[0] == W.SUCCESS
+    assert wq(x2=((64, 128), W.DT_F16), scale=None, x2_strides=(1, 64))[0] == W.SUCCESS   # transposed
+    assert wq(x2=((64, 128), W.DT_F16), scale=None, x2_fmt=W.FORMAT_PACKED)[0] == W.SUCCESS
+    assert wq(x2=((64, 128), W.DT_F16), scale=None, offset=((128,), None))[0] == W.ERR_PARAM_INVALID
+    assert wq(x2=((64, 128), W.DT_F16), scale=None, G=32)[0] == W.ERR_PARAM_INVALID
+    assert wq(x2=((64, 128), W.DT_BF16))[0] == W.ERR_PARAM_INVALID                 # bf16 weight, f16 x1
+    assert wq(x2=((64, 128), W.DT_BF16), scale=None)[0] == W.ERR_PARAM_NULLPTR     # then a scale is required
+    assert wq(x2=((64, 128), W.DT_I8), scale=None)[0] == W.ERR_PARAM_NULLPTR
+    assert wq(x2=((64, 100), W.DT_F16), scale=None)[0] == W.ERR_PARAM_INVALID      # n % 32
+    st, nbytes = W.wqmm_pack_weight_size(T((64, 128), W.DT_BF16), 0)
+    assert st == W.SUCCESS and nbytes == 64 * 128 * 2
+    assert W.wqmm_pack_weight_size(T((64, 128), W.DT_BF16), 1)[0] == W.ERR_PARAM_INVALID  # int8 GEMM tiling
 
 
 def test_attribute_rules():
@@ -232,7 +251,9 @@ def test_pack_size_queries():
     assert st == W.SUCCESS and nb == 8192 * 1024
     st, nb = W.wqmm_pack_weight_size(T((96, 160), W.DT_I8))
     assert st == W.SUCCESS and nb == 2 * 2 * 8192                                   # 2 n-blocks x 2 k-tiles, padded
-    st, _ = W.wqmm_pack_weight_size(T((64, 128), W.DT_F16))
+    st, nb = W.wqmm_pack_weight_size(T((64, 128), W.DT_F16))                  # non-quantised 16-bit weight
+    assert st == W.SUCCESS and nb == 64 * 128 * 2
+    st, _ = W.wqmm_pack_weight_size(T((64, 128), W.DT_F32))
     assert st == W.ERR_PARAM_INVALID
 
 
@@ -246,9 +267,13 @@ def test_pack_size_queries():
     (300, 512, 256),       # wide tiles, fewer than the CTAs: two-step units
     (200, 448, 384),       # odd k-step count
 ])
-def test_schedule_mirror_matches_library_workspace(m, k, n):
+@pytest.mark.parametrize("nonquant", [False, True], ids=["int4", "nonquant"])
+def test_schedule_mirror_matches_library_workspace(m, k, n, nonquant):
     import bench
-    st, ws = wq(x1=((m, k), W.DT_BF16), x2=((k, n), W.DT_I4), scale=((n,), None), x2_fmt=W.FORMAT_PACKED)
+    if nonquant:  # 16-bit weights: the general kernel at every m
+        st, ws = wq(x1=((m, k), W.DT_BF16), x2=((k, n), W.DT_BF16), scale=None, x2_fmt=W.FORMAT_PACKED)
+    else:
+        st, ws = wq(x1=((m, k), W.DT_BF16), x2=((k, n), W.DT_I4), scale=((n,), None), x2_fmt=W.FORMAT_PACKED)
     assert st == W.SUCCESS
     sms = 148  # phase 1 without a GPU plans for a B200
     try:
@@ -257,6 +282,6 @@ def test_schedule_mirror_matches_library_workspace(m, k, n):
             sms = torch.cuda.get_device_properties(0).multi_processor_count
     except ImportError:
         pass
-    s = bench.wqmm_schedule(m, n, k, sms)
+    s = bench.wqmm_schedule(m, n, k, sms, nonquant=nonquant)
     rnd = lambda b: -(-b // 256) * 256
     assert ws == rnd(s["partial_bytes"]) + rnd(s["flag_bytes"]), (s, ws)

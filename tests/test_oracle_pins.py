@@ -324,6 +324,39 @@ def test_int4_zero_offset_unit_scale_is_plain_matmul():
     np.testing.assert_allclose(ye, ref.numpy(), rtol=0, atol=1e-9)
 
 
+@pytest.mark.parametrize("act,transposed", [("bf16", False), ("f16", False), ("bf16", True)])
+def test_non_quantised_is_torch_fp64_matmul(act, transposed):
+    # the non-quantised scenario (x2 of the x1 dtype, no antiquant factors):
+    # out = x1 @ x2 + bias + x3, pinned against torch's float64 matmul on
+    # values decoded by the test's own code
+    case = W.make_wqmm_case(x1_shape=(2, 5, 96), n=48, act=act, wdt=act, x2_transposed=transposed, seed=21)
+    assert case.mode == "none" and case.scale is None and case.offset is None
+    ye, yr = oracle.wqmm(case)
+    w = dec_act(case.x2, act)
+    w = w.T if transposed else w
+    ref = (torch.from_numpy(dec_act(case.x1, act).reshape(case.m, case.k)) @ torch.from_numpy(w)
+           + torch.from_numpy(dec_act(case.bias, act)) + torch.from_numpy(dec_act(case.x3, act).reshape(case.m, case.n)))
+    np.testing.assert_allclose(ye, ref.numpy(), rtol=0, atol=1e-12)
+    # one rounding of the exact value: within half an ulp of the format
+    got = dec_act(yr, act)
+    ulp = np.exp2(np.floor(np.log2(np.abs(ye) + 1e-300)) - (10 if act == "f16" else 7))
+    assert (np.abs(got - ye) <= 0.5 * ulp + 1e-300).all()
+
+
+def test_non_quantised_rejects_antiquant_factors_and_mixed_dtypes():
+    case = W.make_wqmm_case(x1_shape=(3, 64), n=32, act="bf16", wdt="bf16", seed=22)
+    args = dict(m=case.m, k=case.k, n=case.n, act="bf16", wdt="bf16", x1=case.x1, x2=case.x2,
+                x2_strides=case.x2_strides,
+                mode="none", group_size=0, scale_strides=(0, 1))
+    one = np.full((case.n,), 0x3F80, dtype=np.uint16)  # bf16 1.0
+    with pytest.raises(ValueError):
+        oracle.wqmm_raw(**args, scale=None, offset=one)             # an offset without a scale
+    with pytest.raises(ValueError):
+        oracle.wqmm_raw(**{**args, "act": "f16"}, scale=None, offset=None)  # x2 of another dtype
+    with pytest.raises(ValueError):
+        oracle.wqmm_raw(**{**args, "wdt": "i8"}, scale=None, offset=None)   # a quantised weight needs a scale
+
+
 def test_identical_group_rows_equal_per_channel():
     g = W.make_wqmm_case(x1_shape=(6, 128), n=32, act="bf16", wdt="i4", mode="group", group_size=32, seed=13)
     c = W.make_wqmm_case(x1_shape=(6, 128), n=32, act="bf16", wdt="i4", mode="channel", seed=13)

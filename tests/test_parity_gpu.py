@@ -117,6 +117,46 @@ def test_wqmm_small_parity(spec):
     check_wqmm(case)
 
 
+# ---------------------------------------------------------------- non-quantised scenario
+# x2 of the x1 dtype, no antiquant factors: out = x1 @ x2 + bias + x3.  The
+# 16-bit weight is re-laid into the packed tiles and copied into the MMA's
+# tensor-memory operand as it is.  Narrow (split k steps), wide and ragged m
+# tiles, a k tail, 3-D x1, no bias/x3, and the transposed storage.
+NONQUANT = [
+    # name, x1_shape, n, act, extras
+    ("nq_bf16_m16_split", (16, 4096), 256, "bf16", {}),
+    ("nq_f16_m40_ktail", (40, 320), 192, "f16", {}),
+    ("nq_bf16_m300", (300, 512), 384, "bf16", {}),
+    ("nq_f16_m200_transposed", (200, 256), 256, "f16", {"x2_transposed": True}),
+    ("nq_bf16_3d", (2, 9, 256), 128, "bf16", {}),
+    ("nq_f16_nobias_nox3", (64, 128), 128, "f16", {"bias": False, "x3": False}),
+    ("nq_bf16_k96", (24, 96), 160, "bf16", {}),
+]
+
+
+@pytest.mark.parametrize("pack", [True, False], ids=["prepacked", "nd"])
+@pytest.mark.parametrize("spec", NONQUANT, ids=[s[0] for s in NONQUANT])
+def test_wqmm_non_quantised_parity(spec, pack):
+    name, x1s, n, act, extra = spec
+    case = WL.make_wqmm_case(name=name, x1_shape=x1s, n=n, act=act, wdt=act, seed=zlib.crc32(name.encode()) % 10000,
+                             **extra)
+    assert case.scale is None
+    check_wqmm(case, pack=pack)
+
+
+def test_pack_kernel_16bit_layout():
+    # chunk c (k values 8c .. 8c+7 of the tile) of column r at (c * 128 + r) * 16
+    case = WL.make_wqmm_case(x1_shape=(1, 128), n=192, act="bf16", wdt="bf16", seed=7)
+    d = C.wqmm_to_device(case, pack=True)
+    torch.cuda.synchronize()
+    got = d.packed.cpu().numpy().view(np.uint16)
+    k, n = 128, 192
+    w = np.zeros((256, 128), dtype=np.uint16)  # (n padded to 2 blocks, k)
+    w[:n, :k] = case.x2.T
+    want = w.reshape(2, 128, 2, 8, 8).transpose(0, 2, 3, 1, 4).reshape(-1)  # (nb, kt, c, r, 8)
+    assert np.array_equal(got, want)
+
+
 # ---------------------------------------------------------------- small m (m <= 32)
 # The small-m kernel: dequantisation groups that issue their own MMAs, x1
 # fetched per turn by the groups, per-group scale/offset rows staged with the
@@ -542,7 +582,7 @@ def _sample(m, n, nr, nc, seed):
     return rows, cols
 
 
-@pytest.mark.parametrize("name", WL.WORKLOAD_NAMES[:4])
+@pytest.mark.parametrize("name", [nm for nm in WL.WORKLOAD_NAMES if not nm.startswith("w8a8")])
 def test_full_size_workload_sampled(name):
     case = WL.workload(name)
     rows, cols = _sample(case.m, case.n, 96, 768, 1)
@@ -550,7 +590,7 @@ def test_full_size_workload_sampled(name):
 
 
 def test_full_size_int8_workload_sampled():
-    case = WL.workload(WL.WORKLOAD_NAMES[4])
+    case = WL.workload("w8a8_pertoken_4x2048x8192x1024")
     d = C.qmm_to_device(case)
     acc = torch.empty((case.m, case.n), dtype=torch.int32, device="cuda")
     C.qmm_call(d, raw_acc=acc)

@@ -18,7 +18,7 @@ from . import (DT_BF16, DT_F16, DT_F32, DT_FP8E4M3, DT_I4, DT_I8, DT_I32, FORMAT
                wqmm_executor_destroy, wqmm_get_workspace_size, wqmm_run)
 
 _ACT = {"f16": DT_F16, "bf16": DT_BF16}
-_WDT = {"i8": DT_I8, "i4": DT_I4, "fp8": DT_FP8E4M3}
+_WDT = {"i8": DT_I8, "i4": DT_I4, "fp8": DT_FP8E4M3, "f16": DT_F16, "bf16": DT_BF16}  # f16/bf16: non-quantised
 
 
 def _torch():
@@ -61,16 +61,21 @@ def wqmm_to_device(case, device="cuda", pack=True, stream=None) -> WqmmDevice:
     torch = _torch()
     k, n = case.k, case.n
     x1 = _act_view(_dev(case.x1.view(np.int16), device), case.act).reshape(case.x1_shape)
-    x2s = _dev(case.x2.view(np.uint8) if case.x2.dtype != np.int8 else case.x2, device)
+    if case.wdt in ("f16", "bf16"):
+        x2s = _dev(case.x2.view(np.int16), device)
+    else:
+        x2s = _dev(case.x2.view(np.uint8) if case.x2.dtype != np.int8 else case.x2, device)
     strides = (1, k) if case.x2_transposed else (n, 1)
     x2d = desc(data=x2s.data_ptr(), dtype=_WDT[case.wdt], shape=(k, n), strides=strides)
     packed = None
     if pack and k > 0:
         packed, x2d = pack_weight(x2d, False, stream)
-    sshape = tuple(case.scale_shape)
-    sc = _act_view(_dev(case.scale.view(np.int16), device), case.act)
+    sshape = None if case.scale is None else tuple(case.scale_shape)
+    sc = None if case.scale is None else _act_view(_dev(case.scale.view(np.int16), device), case.act)
     of = None if case.offset is None else _act_view(_dev(case.offset.view(np.int16), device), case.act)
-    if case.mode == "group" and case.scale_transposed:
+    if sc is None:
+        pass
+    elif case.mode == "group" and case.scale_transposed:
         ng = sshape[0]
         sc = sc.reshape(n, ng).t()
         of = None if of is None else of.reshape(n, ng).t()
@@ -80,7 +85,7 @@ def wqmm_to_device(case, device="cuda", pack=True, stream=None) -> WqmmDevice:
     bias = None if case.bias is None else _act_view(_dev(case.bias.view(np.int16), device), case.act)
     x3 = None if case.x3 is None else _act_view(_dev(case.x3.view(np.int16), device), case.act).reshape(case.out_shape)
     out = torch.empty(case.out_shape, dtype=x1.dtype, device=device)
-    return WqmmDevice(x1=x1, x2=x2s, x2_desc=x2d, scale=sc, scale_desc=desc(sc), offset=of,
+    return WqmmDevice(x1=x1, x2=x2s, x2_desc=x2d, scale=sc, scale_desc=None if sc is None else desc(sc), offset=of,
                       offset_desc=None if of is None else desc(of), bias=bias, x3=x3, out=out,
                       group_size=case.group_size, packed=packed)
 

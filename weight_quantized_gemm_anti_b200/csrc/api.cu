@@ -149,6 +149,17 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 bool act_dtype_ok(int dt) { return dt == WQMM_DT_F16 || dt == WQMM_DT_BF16; }
 
+// The anti-quant GEMM's weight kind for an x2 dtype (float16 / bfloat16: the
+// non-quantised scenario, x2 of the x1 dtype).
+int weight_kind(int x2_dtype) {
+  switch (x2_dtype) {
+    case WQMM_DT_I4: return kW4;
+    case WQMM_DT_I8: return kW8;
+    case WQMM_DT_FP8E4M3: return kWFp8;
+    default: return kWH;
+  }
+}
+
 const char* dt_name(int dt) {
   switch (dt) {
     case WQMM_DT_F16: return "float16";
@@ -250,7 +261,7 @@ uint64_t packed_bytes_for(int x2_dtype, int64_t k, int64_t n, bool for_qmm) {
     const uint64_t nb = (n + kQNBlock - 1) / kQNBlock, kt = (k + kQKTile - 1) / kQKTile;
     return nb * kt * kQTileBytes;
   }
-  const int wk = x2_dtype == WQMM_DT_I4 ? kW4 : (x2_dtype == WQMM_DT_I8 ? kW8 : kWFp8);
+  const int wk = weight_kind(x2_dtype);
   const uint64_t nb = (n + kWqNBlock - 1) / kWqNBlock, kt = (k + kWqKTile - 1) / kWqKTile;
   return nb * kt * wq_tile_bytes(wk);
 }
@@ -316,9 +327,12 @@ extern "C" wqmm_status wqmm_get_workspace_size(const wqmm_tensor* x1, const wqmm
                                                const wqmm_tensor* output, uint64_t* workspace_size,
                                                wqmm_executor** executor) {
   (void)group;  // communication domain: unused for one rank
-  // ---- CheckNotNull
-  if (!x1 || !x2 || !scale || !output)
-    return fail(WQMM_ERR_PARAM_NULLPTR, "x1, x2, antiquantScale and output must not be null");
+  // ---- CheckNotNull (antiquantScale may be null only in the non-quantised
+  // scenario, x2 of the x1 dtype)
+  if (!x1 || !x2 || !output) return fail(WQMM_ERR_PARAM_NULLPTR, "x1, x2 and output must not be null");
+  const bool nonquant = act_dtype_ok(x1->dtype) && x2->dtype == x1->dtype;
+  if (!scale && !nonquant)
+    return fail(WQMM_ERR_PARAM_NULLPTR, "antiquantScale must not be null for int8, int4 or float8_e4m3fn weights");
   if (!reduce_op) return fail(WQMM_ERR_PARAM_NULLPTR, "reduceOp must not be null");
   if (!workspace_size || !executor) return fail(WQMM_ERR_PARAM_NULLPTR, "workspaceSize and executor must not be null");
   *executor = nullptr;
@@ -337,8 +351,12 @@ extern "C" wqmm_status wqmm_get_workspace_size(const wqmm_tensor* x1, const wqmm
   const int adt = x1->dtype;
   if (!act_dtype_ok(adt))
     return fail(WQMM_ERR_PARAM_INVALID, "x1 dtype %s not supported (float16, bfloat16)", dt_name(adt));
-  if (x2->dtype != WQMM_DT_I8 && x2->dtype != WQMM_DT_I4 && x2->dtype != WQMM_DT_FP8E4M3)
-    return fail(WQMM_ERR_PARAM_INVALID, "x2 dtype %s not supported (int8, int4, float8_e4m3fn)", dt_name(x2->dtype));
+  if (x2->dtype != WQMM_DT_I8 && x2->dtype != WQMM_DT_I4 && x2->dtype != WQMM_DT_FP8E4M3 && !nonquant)
+    return fail(WQMM_ERR_PARAM_INVALID, "x2 dtype %s not supported (int8, int4, float8_e4m3fn, or the x1 dtype)",
+                dt_name(x2->dtype));
+  if (nonquant && (scale || offset))
+    return fail(WQMM_ERR_PARAM_INVALID,
+                "x2 of the x1 dtype (non-quantised) takes no antiquantScale or antiquantOffset");
   const wqmm_tensor* same[] = {scale, offset, bias, x3, output};
   const char* same_names[] = {"antiquantScale", "antiquantOffset", "bias", "x3", "output"};
   for (int i = 0; i < 5; ++i)
@@ -358,6 +376,8 @@ extern "C" wqmm_status wqmm_get_workspace_size(const wqmm_tensor* x1, const wqmm
                   (long long)group_size, (long long)hi);
   }
   if (group_size < 0) return fail(WQMM_ERR_PARAM_INVALID, "antiquantGroupSize must not be negative");
+  if (nonquant && group_size != 0)
+    return fail(WQMM_ERR_PARAM_INVALID, "antiquantGroupSize must be 0 for x2 of the x1 dtype (non-quantised)");
   if (x2->dtype == WQMM_DT_FP8E4M3 && offset)
     return fail(WQMM_ERR_PARAM_INVALID, "antiquantOffset must be null for float8_e4m3fn weights");
 
@@ -380,7 +400,9 @@ extern "C" wqmm_status wqmm_get_workspace_size(const wqmm_tensor* x1, const wqmm
   int mode;
   int64_t ng = 0;
   bool scale_t = false;
-  if (group_size != 0 && k != 0) {
+  if (nonquant) {
+    mode = kNoQuant;
+  } else if (group_size != 0 && k != 0) {
     mode = kPerGroup;
     ng = (k + group_size - 1) / group_size;
     if (scale->ndim != 2 || scale->shape[0] != ng || scale->shape[1] != n)
@@ -452,7 +474,7 @@ extern "C" wqmm_status wqmm_get_workspace_size(const wqmm_tensor* x1, const wqmm
   ex->out = output->data;
   ex->bias = bias ? bias->data : nullptr;
   ex->x3 = x3 ? x3->data : nullptr;
-  ex->scale = scale->data;
+  ex->scale = scale ? scale->data : nullptr;
   ex->offset = offset ? offset->data : nullptr;
   ex->scale_transposed = scale_t;
   ex->mode = mode;
@@ -493,7 +515,8 @@ extern "C" wqmm_status wqmm_get_workspace_size(const wqmm_tensor* x1, const wqmm
     // get several), unless WQMM_STREAMK=0 asks for whole tiles.
     {
       const char* sm_env = std::getenv("WQMM_SMALLM");
-      ex->smallm = (ex->bn == 16 || ex->bn == 32) && !(sm_env && std::atoi(sm_env) == 0) ? 1 : 0;
+      // (16-bit weights, the non-quantised scenario, run on the general kernel)
+      ex->smallm = (ex->bn == 16 || ex->bn == 32) && !nonquant && !(sm_env && std::atoi(sm_env) == 0) ? 1 : 0;
     }
     if (ex->smallm && !forbid_sk) {
       // units of two k steps when the step count is even: the kernel then takes
@@ -578,7 +601,7 @@ extern "C" wqmm_status wqmm_get_workspace_size(const wqmm_tensor* x1, const wqmm
     // 141.3 us) and not for int8 (W8A16 2048x4096x4096: 94.3 vs 92.2 us): the
     // default for int4 at 256 rows; WQMM_PAIR=1 / 0 forces them on / off.
     const char* pair_env = std::getenv("WQMM_PAIR");
-    const int wk = x2->dtype == WQMM_DT_I4 ? kW4 : (x2->dtype == WQMM_DT_I8 ? kW8 : kWFp8);
+    const int wk = weight_kind(x2->dtype);
     const bool want_pair = pair_env ? std::atoi(pair_env) == 1 : (ex->bn == 256 && wk == kW4);
     if (!ex->smallm && !ex->stream_k && want_pair && (ex->bn == 192 || ex->bn == 256) && num_nb >= 2) {
       const int ps = pair_slots(ex->bn, wk, adt == WQMM_DT_BF16);
@@ -801,7 +824,7 @@ wqmm_status check_workspace(const wqmm_executor* ex, void* ws, uint64_t size) {
 wqmm_status run_wqmm(void* ws, wqmm_executor* ex, cudaStream_t s) {
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   const bool bf16 = ex->act_dtype == WQMM_DT_BF16;
-  const int wk = ex->x2_dtype == WQMM_DT_I4 ? kW4 : (ex->x2_dtype == WQMM_DT_I8 ? kW8 : kWFp8);
+  const int wk = weight_kind(ex->x2_dtype);
   cudaError_t e;
   if (ex->k == 0) {
     EpiParams ep{};
@@ -1011,7 +1034,8 @@ wqmm_status check_pack_args(const wqmm_tensor* x2, int32_t for_qmm, bool* transp
   if (x2->ndim != 2) return fail(WQMM_ERR_PARAM_INVALID, "x2 must be 2-D (k, n)");
   if (for_qmm) {
     if (x2->dtype != WQMM_DT_I8) return fail(WQMM_ERR_PARAM_INVALID, "the int8 GEMM packs int8 weights only");
-  } else if (x2->dtype != WQMM_DT_I8 && x2->dtype != WQMM_DT_I4 && x2->dtype != WQMM_DT_FP8E4M3) {
+  } else if (x2->dtype != WQMM_DT_I8 && x2->dtype != WQMM_DT_I4 && x2->dtype != WQMM_DT_FP8E4M3 &&
+             !act_dtype_ok(x2->dtype)) {
     return fail(WQMM_ERR_PARAM_INVALID, "x2 dtype %s cannot be packed", dt_name(x2->dtype));
   }
   const int64_t k = x2->shape[0], n = x2->shape[1];
@@ -1046,7 +1070,7 @@ extern "C" wqmm_status wqmm_pack_weight(const wqmm_tensor* x2, int32_t for_int8_
   pp.n = static_cast<int>(x2->shape[1]);
   pp.s0 = t ? 1 : pp.n;
   pp.s1 = t ? pp.k : 1;
-  pp.wk = x2->dtype == WQMM_DT_I4 ? kW4 : (x2->dtype == WQMM_DT_I8 ? kW8 : kWFp8);
+  pp.wk = weight_kind(x2->dtype);
   pp.for_qmm = for_int8_gemm != 0;
   cudaError_t e = launch_pack(pp, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "weight pack launch");

@@ -7,17 +7,21 @@
 
 namespace wqmm {
 
-// Weight kinds of the anti-quant GEMM.
-enum WeightKind : int { kW4 = 0, kW8 = 1, kWFp8 = 2 };
-// Scale / offset modes ("计算公式" symbol table: per-tensor, per-channel, per-group).
-enum QuantMode : int { kPerTensor = 0, kPerChannel = 1, kPerGroup = 2 };
+// Weight kinds of the anti-quant GEMM; kWH: a float16/bfloat16 weight of the
+// activations' own type (the non-quantised scenario: no scale, no offset).
+enum WeightKind : int { kW4 = 0, kW8 = 1, kWFp8 = 2, kWH = 3 };
+// Scale / offset modes ("计算公式" symbol table: per-tensor, per-channel,
+// per-group); kNoQuant: no antiquantScale / antiquantOffset at all.
+enum QuantMode : int { kPerTensor = 0, kPerChannel = 1, kPerGroup = 2, kNoQuant = 3 };
 
 // Packed weight geometry for the anti-quant GEMM: tiles of 128 n-rows x 64 k,
 // tile (nb, kt) at byte ((nb * KT + kt) * tile_bytes); inside a tile, 16-byte
 // chunk c of row r sits at ((c * 128 + r) * 16).
 constexpr int kWqNBlock = 128;
 constexpr int kWqKTile = 64;
-__host__ __device__ constexpr int wq_tile_bytes(int wk) { return wk == kW4 ? 4096 : 8192; }
+__host__ __device__ constexpr int wq_tile_bytes(int wk) { return wk == kW4 ? 4096 : (wk == kWH ? 16384 : 8192); }
+// 16-byte chunks per weight column of one packed tile (64 k values)
+__host__ __device__ constexpr int wq_chunks_per_col(int wk) { return wq_tile_bytes(wk) / (kWqNBlock * 16); }
 // Packed weight geometry for the int8 GEMM: tiles of 256 n-rows x 128 k bytes,
 // 32 KB each, stored in the 128-byte-swizzled K-major order (16-byte chunk c of
 // row r at r * 128 + ((c ^ (r & 7)) * 16)).

@@ -15,16 +15,18 @@ namespace wqmm {
 __device__ uint32_t g_device_error = 0;
 
 // ---------------------------------------------------------------- weight pack
-// Read one logical weight element (kk, nn) of x2 as its raw integer code:
-// int8 / fp8 byte, or the 4-bit two's-complement nibble (even linear index in
-// the low nibble).  Out-of-range elements read as 0.
-__device__ __forceinline__ int read_code(const PackParams& p, int kk, int nn) {
+// Read one logical weight element (kk, nn) of x2 as its raw code: int8 / fp8
+// byte, the 4-bit two's-complement nibble (even linear index in the low
+// nibble), or the 16-bit float16/bfloat16 pattern.  Out-of-range elements read
+// as 0.
+__device__ __forceinline__ uint32_t read_code(const PackParams& p, int kk, int nn) {
   if (kk >= p.k || nn >= p.n) return 0;
   const int64_t idx = static_cast<int64_t>(kk) * p.s0 + static_cast<int64_t>(nn) * p.s1;
   if (p.wk == kW4) {
     const uint8_t b = p.src[idx >> 1];
     return (idx & 1) ? (b >> 4) : (b & 0xF);
   }
+  if (p.wk == kWH) return reinterpret_cast<const uint16_t*>(p.src)[idx];
   return p.src[idx];
 }
 
@@ -34,9 +36,10 @@ __device__ __forceinline__ int read_code(const PackParams& p, int kk, int nn) {
 // 0x6400 (f16 1024.0) exponent pattern gives 128+q+8 / 1024+q+8 exactly.
 // int8 chunk (16 k values): byte b = k0 + b, stored biased as (q + 128).
 // fp8 chunk: byte b = k0 + b, raw e4m3 code.
+// 16-bit chunk (8 k values): half-word h = k0 + h, the value's own bits.
 __global__ void pack_wq_kernel(PackParams p, int64_t total_chunks) {
-  const int chunks_per_row = (p.wk == kW4) ? 2 : 4;
-  const int vals_per_chunk = (p.wk == kW4) ? 32 : 16;
+  const int chunks_per_row = wq_chunks_per_col(p.wk);
+  const int vals_per_chunk = kWqKTile / chunks_per_row;
   const int kt_total = (p.k + kWqKTile - 1) / kWqKTile;
   for (int64_t g = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; g < total_chunks;
        g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -60,6 +63,8 @@ __global__ void pack_wq_kernel(PackParams p, int64_t total_chunks) {
         }
         words[w] = word;
       }
+    } else if (p.wk == kWH) {
+      for (int w = 0; w < 4; ++w) words[w] = read_code(p, k0 + 2 * w, nn) | (read_code(p, k0 + 2 * w + 1, nn) << 16);
     } else {
       const uint32_t bias = (p.wk == kW8) ? 0x80u : 0u;
       for (int w = 0; w < 4; ++w) {
@@ -114,7 +119,7 @@ cudaError_t launch_pack(const PackParams& p, cudaStream_t s) {
     pack_q_kernel<<<grid_for(total, 256), 256, 0, s>>>(p, total);
   } else {
     const int64_t nb = (p.n + kWqNBlock - 1) / kWqNBlock, kt = (p.k + kWqKTile - 1) / kWqKTile;
-    const int64_t total = nb * kt * ((p.wk == kW4) ? 2 : 4) * kWqNBlock;
+    const int64_t total = nb * kt * wq_chunks_per_col(p.wk) * kWqNBlock;
     pack_wq_kernel<<<grid_for(total, 256), 256, 0, s>>>(p, total);
   }
   return cudaGetLastError();
@@ -160,7 +165,7 @@ __device__ __forceinline__ uint16_t f32_to_act(float v, int bf16) {
 __device__ __forceinline__ bool small_int_offset(float off) { return off == rintf(off) && fabsf(off) <= 112.f; }
 
 __device__ __forceinline__ float epilogue_scale(const EpiParams& p, int nn) {
-  if (p.mode == kPerGroup) return 1.f;
+  if (p.mode == kPerGroup || p.mode == kNoQuant) return 1.f;
   const int i = (p.mode == kPerTensor) ? 0 : nn;
   const float s = act_to_f32(p.scale[i], p.act_bf16);
   const float o = p.offset ? act_to_f32(p.offset[i], p.act_bf16) : 0.f;

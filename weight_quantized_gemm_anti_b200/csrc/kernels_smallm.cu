@@ -616,6 +616,7 @@ cudaError_t launch_sm_spg(const WqParams& p, int grid, cudaStream_t s) {
 
 template <int BN>
 cudaError_t launch_sm_bn(const WqParams& p, int wk, bool bf16, int grid, cudaStream_t s) {
+  if (wk == kWH) return cudaErrorInvalidValue;  // 16-bit weights run on the general kernel
   if (wk == kW4) return bf16 ? launch_sm_spg<BN, kW4, true>(p, grid, s) : launch_sm_spg<BN, kW4, false>(p, grid, s);
   if (wk == kW8) return bf16 ? launch_sm_spg<BN, kW8, true>(p, grid, s) : launch_sm_spg<BN, kW8, false>(p, grid, s);
   return bf16 ? launch_sm_spg<BN, kWFp8, true>(p, grid, s) : launch_sm_spg<BN, kWFp8, false>(p, grid, s);

@@ -82,16 +82,26 @@ struct Cfg {
   // tiles the x1 ring gets the depth and 40-48 KB of weights cover theirs.
   // Narrow m tiles stream weights from HBM: the weight ring then takes most of
   // the space, to keep enough bytes in flight.
-  // epilogue staging: kEpiRows output rows x 128 columns, fp32
+  // epilogue staging: per epilogue warp, kEpiRows output rows x its 32
+  // columns, fp32, rows kEpiPitch floats apart (the padding keeps the
+  // row-wise 16-byte reads free of bank conflicts)
   static constexpr int kEpiRows = 16;
-  static constexpr int kStageBytes = kEpiRows * 128 * 4;
+  static constexpr int kEpiPitch = 36;
+  static constexpr int kStageBytes = 4 * kEpiRows * kEpiPitch * 4;
   static constexpr int kSmemBudget = 224 * 1024 - kStageBytes;
   // A weight stage holds kWQ consecutive k steps (16 KB) and is filled by one
   // or two bulk copies: a copy instruction holds its issuing thread for hundreds
   // of cycles whatever its size, so fewer, larger copies stream faster.
   static constexpr int kWQ = 16384 / kTile;
   static constexpr int kWStageBytes = kWQ * kTile;
-  static constexpr int kWStages = BN <= 64 ? cmin(12, (kSmemBudget - 8 * kX1Bytes) / kWStageBytes) : 3;
+  // A parity wait on an mbarrier can only look one phase ahead: the
+  // dequantisation groups' turns of one cycle (DG * SPG steps, DG * SPG / kWQ
+  // stages) must all lie in distinct stages of the weight ring, or a group
+  // would wait for a stage's next fill while the current one is still pending
+  // and see it as complete.
+  static constexpr int kWCycle = DG * SPG / kWQ;
+  static constexpr int kWStages =
+      BN <= 64 ? cmin(12, (kSmemBudget - 8 * kX1Bytes) / kWStageBytes) : cmax(3, kWCycle);
   static constexpr int kXStages = cmin(16, (kSmemBudget - kWStages * kWStageBytes) / kX1Bytes);
   // The MMA issuer waits once per batch of k steps (half the A stages) and then
   // issues the whole batch: every barrier wait in the issuing thread costs the
@@ -104,6 +114,8 @@ struct Cfg {
   static constexpr int kThreads = 32 * (8 + 4 * DG);
   static constexpr int kSmemBytes = kXStages * kX1Bytes + kWStages * kWStageBytes + kStageBytes + 1024;
   static_assert(kAStages >= DG * SPG && kAStages % (DG * SPG) == 0, "A stages");
+  static_assert(kWStages >= kWCycle, "one cycle of dequantisation turns fits in the weight ring");
+  static_assert(kXStages >= DG * SPG, "one cycle of dequantisation turns fits in the x1 ring");
   static_assert(kWQ % SPG == 0 && (DG * SPG) % kWQ == 0, "a group's turn lies in one weight stage; turns cover whole stages");
   static_assert(kACol0 + kAStages * 32 <= 512, "TMEM budget");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -401,20 +413,29 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR, SPG>::kThreads, 1)
     }
   } else if (warp < 6) {
     // ============================================================ epilogue
-    // Per chunk of kEpiRows accumulator columns (output rows): (1) each thread
+    // Each warp drains its own TMEM lane quadrant (32 weight columns) in
+    // chunks of kEpiRows accumulator columns (output rows): (1) each thread
     // reads its weight column's values from TMEM, applies the per-column scale
-    // and writes them, fp32, into a staging tile [row][column]; (2) after a
-    // barrier of the four epilogue warps, each thread takes 8 consecutive
-    // columns of one row: + bias, + x3 (16-byte loads), one rounding, one
-    // 16-byte store.  Both global streams are coalesced whole rows.
+    // and writes them, fp32, into the warp's staging tile [row][column]; (2)
+    // after a __syncwarp, each thread takes 8 consecutive columns of one row:
+    // + bias, + x3 (16-byte loads), one rounding, one 16-byte store (64
+    // contiguous bytes per row and warp).  The next chunk's TMEM load is in
+    // flight during (2), and no barrier couples the four warps, so the
+    // accumulator is handed back to the MMA after BN / kEpiRows short rounds.
     const int quad = warp & 3;
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
     const int et = threadIdx.x - 64;        // 0..127 over warps 2..5
-    const int col8 = (et & 15) * 8;          // phase 2: 8 columns ...
-    const int prow = et >> 4;                // ... of rows prow, prow + 8, ...
+    const int col8 = quad * 32 + (lane & 3) * 8;  // phase 2: 8 columns ...
+    const int prow = lane >> 2;                   // ... of rows prow, prow + 8, ...
     constexpr int kER = C::kEpiRows;
+    constexpr int kEP = C::kEpiPitch;
     constexpr int kPasses = kER / 8;
-    float* stage = reinterpret_cast<float*>(s_stage);
+    static_assert(kER == 16, "the drain loads 16 accumulator columns at a time");
+    // the next chunk's load is issued before phase 2 where registers allow
+    // (512 threads: 128 per thread); the 768-thread kernels load each chunk
+    // in turn
+    constexpr bool kPrefetch = C::kThreads <= 512;
+    float* wst = reinterpret_cast<float*>(s_stage) + quad * (kER * kEP);
     uint32_t j = 0;
     while (walk.next(p, it)) {
       const int ab = j % C::kNAcc;
@@ -481,6 +502,9 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR, SPG>::kThreads, 1)
         __threadfence();
         others = p.partial + sk_r * p.max_slots * (BN * kWqNBlock);  // slot s at others + s * BN * 128
       }
+      const uint32_t acc_addr = tmem + lane_addr + ab * C::kAccCols;
+      uint32_t v[kER];
+      if constexpr (kPrefetch) tmem_ld_x16(acc_addr, v);
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += kER) {
         const bool last = (c0 + kER >= BN);
@@ -494,14 +518,10 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR, SPG>::kThreads, 1)
                        ? *reinterpret_cast<const uint4*>(p.x3 + mm * p.n + nn8)
                        : make_uint4(0u, 0u, 0u, 0u);
         }
-        uint32_t v[kER];
-        if constexpr (kER == 32)
-          tmem_ld_x32(tmem + lane_addr + ab * C::kAccCols + c0, v);
-        else
-          tmem_ld_x16(tmem + lane_addr + ab * C::kAccCols + c0, v);
-        tmem_wait_ld();
+        if constexpr (!kPrefetch) tmem_ld_x16(acc_addr + c0, v);
+        tmem_wait_ld_r16(v);
         if (last) {
-          // the whole accumulator is in registers or staged: hand it back
+          // the whole accumulator has been read: hand it back
           tc_fence_before();
           __syncwarp();
           if (lane == 0) arrive_mma_cta(&bar_accempty[ab]);
@@ -509,6 +529,7 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR, SPG>::kThreads, 1)
         if (part) {
 #pragma unroll
           for (int q = 0; q < kER; ++q) part[(c0 + q) * kWqNBlock + nl] = __uint_as_float(v[q]);
+          if (kPrefetch && !last) tmem_ld_x16(acc_addr + c0 + kER, v);
           continue;
         }
         if (others) {
@@ -522,19 +543,21 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR, SPG>::kThreads, 1)
             for (int q = 0; q < kER; ++q) acc[q] += src[q * kWqNBlock];
           }
 #pragma unroll
-          for (int q = 0; q < kER; ++q) stage[q * kWqNBlock + nl] = acc[q] * escale;
+          for (int q = 0; q < kER; ++q) wst[q * kEP + lane] = acc[q] * escale;
         } else {
 #pragma unroll
-          for (int q = 0; q < kER; ++q) stage[q * kWqNBlock + nl] = __uint_as_float(v[q]) * escale;
+          for (int q = 0; q < kER; ++q) wst[q * kEP + lane] = __uint_as_float(v[q]) * escale;
         }
-        named_bar_sync(1, 128);
+        __syncwarp();
+        if (kPrefetch && !last) tmem_ld_x16(acc_addr + c0 + kER, v);  // in flight during phase 2
 #pragma unroll
         for (int ps = 0; ps < kPasses; ++ps) {
           const int row = ps * 8 + prow;
           const int64_t mm = m0 + c0 + row;
           if (col8_ok && mm < p.m) {
-            const float4 lo = *reinterpret_cast<const float4*>(stage + row * kWqNBlock + col8);
-            const float4 hi = *reinterpret_cast<const float4*>(stage + row * kWqNBlock + col8 + 4);
+            const float* src = wst + row * kEP + (lane & 3) * 8;
+            const float4 lo = *reinterpret_cast<const float4*>(src);
+            const float4 hi = *reinterpret_cast<const float4*>(src + 4);
             const float y[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
             const uint32_t xw[4] = {xv[ps].x, xv[ps].y, xv[ps].z, xv[ps].w};
             uint32_t o[4];
@@ -547,7 +570,7 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR, SPG>::kThreads, 1)
             *reinterpret_cast<uint4*>(p.out + mm * p.n + nn8) = make_uint4(o[0], o[1], o[2], o[3]);
           }
         }
-        named_bar_sync(1, 128);  // the staging tile is rewritten by the next chunk
+        __syncwarp();  // the staging tile is rewritten by the next chunk
       }
       if (part && p.sk_inline) {
         // this owner's partial is complete: publish it to the tile's first owner
@@ -616,7 +639,7 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR, SPG>::kThreads, 1)
           live = false;
           break;
         }
-        constexpr int kChunks = (WK == kW4) ? 2 : 4;
+        constexpr int kChunks = wq_chunks_per_col(WK);
         uint4 ch[SPG][kChunks];
 #pragma unroll
         for (int j = 0; j < SPG; ++j) {
@@ -655,6 +678,15 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR, SPG>::kThreads, 1)
             } else {
               dq4_general<BF16>(ch[j][0], cc.off, cc.s, a);
               dq4_general<BF16>(ch[j][1], cc.off, cc.s, a + 16);
+            }
+          } else if constexpr (WK == kWH) {
+            // non-quantised: the weight is already in the MMA's operand type
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c) {
+              a[4 * c] = ch[j][c].x;
+              a[4 * c + 1] = ch[j][c].y;
+              a[4 * c + 2] = ch[j][c].z;
+              a[4 * c + 3] = ch[j][c].w;
             }
           } else if constexpr (WK == kW8) {
             if constexpr (GRP) {
@@ -795,7 +827,7 @@ constexpr int dgroups() {
 template <int BN, bool PAIR, int WK, bool BF16, int SPG>
 cudaError_t launch_spg(const CUtensorMap& tmap, const WqParams& p, int grid, cudaStream_t s) {
   constexpr int DG = SPG == 2 ? 2 : dgroups<BN>();
-  if constexpr (WK == kWFp8) {  // fp8 weights have per-channel scales only
+  if constexpr (WK == kWFp8 || WK == kWH) {  // fp8: per-channel scales only; 16-bit: none
     return launch_one<BN, DG, WK, BF16, PAIR, false, SPG>(tmap, p, grid, s);
   } else {
     return p.mode == kPerGroup ? launch_one<BN, DG, WK, BF16, PAIR, true, SPG>(tmap, p, grid, s)
@@ -805,7 +837,7 @@ cudaError_t launch_spg(const CUtensorMap& tmap, const WqParams& p, int grid, cud
 
 template <int BN, bool PAIR, int WK, bool BF16>
 cudaError_t launch_mode(const CUtensorMap& tmap, const WqParams& p, int grid, cudaStream_t s) {
-  if constexpr (BN >= 128 && !PAIR) {
+  if constexpr (BN >= 128 && !PAIR && WK != kWH) {  // a 16-bit step fills a whole weight stage
     if (p.kt_total % 2 == 0 && (!p.stream_k || p.sk_unit == 2))
       return launch_spg<BN, PAIR, WK, BF16, 2>(tmap, p, grid, s);
   }
@@ -818,6 +850,14 @@ cudaError_t launch_bn(const CUtensorMap& tmap, const WqParams& p, int wk, bool b
     return bf16 ? launch_mode<BN, PAIR, kW4, true>(tmap, p, grid, s) : launch_mode<BN, PAIR, kW4, false>(tmap, p, grid, s);
   if (wk == kW8)
     return bf16 ? launch_mode<BN, PAIR, kW8, true>(tmap, p, grid, s) : launch_mode<BN, PAIR, kW8, false>(tmap, p, grid, s);
+  if (wk == kWH) {
+    if constexpr (PAIR) {
+      return cudaErrorInvalidValue;  // no pair mode for 16-bit weights
+    } else {
+      return bf16 ? launch_mode<BN, false, kWH, true>(tmap, p, grid, s)
+                  : launch_mode<BN, false, kWH, false>(tmap, p, grid, s);
+    }
+  }
   return bf16 ? launch_mode<BN, PAIR, kWFp8, true>(tmap, p, grid, s)
               : launch_mode<BN, PAIR, kWFp8, false>(tmap, p, grid, s);
 }
@@ -863,7 +903,7 @@ __global__ void __launch_bounds__(256) wqmm_fixup_kernel(const FixupParams p) {
     float escale[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) escale[e] = 1.f;
-    if (p.mode != kPerGroup) {
+    if (p.mode == kPerTensor || p.mode == kPerChannel) {
       bool small = true;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -922,6 +962,7 @@ int pair_slots_bn(int wk, bool act_bf16) {
   constexpr int DG = dgroups<BN>();
   if (wk == kW4) return act_bf16 ? pair_slots_one<BN, DG, kW4, true>() : pair_slots_one<BN, DG, kW4, false>();
   if (wk == kW8) return act_bf16 ? pair_slots_one<BN, DG, kW8, true>() : pair_slots_one<BN, DG, kW8, false>();
+  if (wk == kWH) return 0;
   return act_bf16 ? pair_slots_one<BN, DG, kWFp8, true>() : pair_slots_one<BN, DG, kWFp8, false>();
 }
 

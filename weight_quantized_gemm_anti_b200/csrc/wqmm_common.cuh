@@ -349,6 +349,13 @@ struct ColConst {
 template <bool BF16, int WK>
 __device__ __forceinline__ ColConst col_const(const WqParams& p, int nn, bool col_ok) {
   ColConst c;
+  if constexpr (WK == kWH) {  // non-quantised: no scale, no offset
+    c.s = 1.f;
+    c.off = 0.f;
+    c.c2 = 0u;
+    c.fast = true;
+    return c;
+  }
   const int idx = (p.mode == kPerTensor) ? 0 : (col_ok ? nn : 0);
   c.s = act_f32(p.scale[idx], BF16);
   c.off = p.offset ? act_f32(p.offset[idx], BF16) : 0.f;

@@ -80,13 +80,13 @@ class WqmmCase:
     k: int
     n: int
     act: str                           # "f16" | "bf16"
-    wdt: str                           # "i8" | "i4" | "fp8"
-    mode: str                          # "tensor" | "channel" | "group"
+    wdt: str                           # "i8" | "i4" | "fp8"; == act: non-quantised
+    mode: str                          # "tensor" | "channel" | "group" | "none"
     group_size: int
     x1: np.ndarray
     x2: np.ndarray                     # storage, see module docstring
     x2_transposed: bool
-    scale: np.ndarray
+    scale: Optional[np.ndarray]        # None in the non-quantised scenario
     offset: Optional[np.ndarray]
     bias: Optional[np.ndarray]
     x3: Optional[np.ndarray]
@@ -114,6 +114,8 @@ class WqmmCase:
     @property
     def scale_strides(self) -> Tuple[int, int]:
         """Element strides of scale viewed as (rows, n)."""
+        if self.mode == "none":
+            return (0, 0)
         if self.mode == "group":
             ng = self.scale_shape[0]
             return (1, ng) if self.scale_transposed else (self.n, 1)
@@ -167,7 +169,9 @@ def make_wqmm_case(*, name="case", x1_shape=(16, 256), n=128, act="bf16", wdt="i
     int4 [-8,7]) or over all finite fp8-e4m3 codes; scale ~ U[scale_range];
     offset ~ integer U[offset_range] (or U[a,b] continuous with
     ``fractional_offset``); bias, x3 ~ N(0,1). ``scale_const``/``offset_const``
-    give per-tensor constants instead of draws."""
+    give per-tensor constants instead of draws.  ``wdt`` equal to ``act`` is
+    the non-quantised scenario: x2 ~ N(0, 0.05^2) in the activation format, no
+    scale or offset (``mode`` "none")."""
     r = _rngs(seed)
     k = x1_shape[-1]
     m = int(np.prod(x1_shape[:-1]))
@@ -182,10 +186,16 @@ def make_wqmm_case(*, name="case", x1_shape=(16, 256), n=128, act="bf16", wdt="i
     elif wdt == "fp8":
         c = e4m3_bits_from_codes(r["x2"], (k, n))
         x2 = np.ascontiguousarray(c.T) if x2_transposed else c
+    elif wdt == act:
+        w = act_bits(0.05 * r["x2"].standard_normal(size=(k, n)), act)
+        x2 = np.ascontiguousarray(w.T) if x2_transposed else w
+        mode = "none"
     else:
         raise ValueError(wdt)
 
-    if mode == "tensor":
+    if mode == "none":
+        sshape = None
+    elif mode == "tensor":
         sshape = (1,)
     elif mode == "channel":
         sshape = (1, n) if scale_2d else (n,)
@@ -195,11 +205,13 @@ def make_wqmm_case(*, name="case", x1_shape=(16, 256), n=128, act="bf16", wdt="i
     else:
         raise ValueError(mode)
 
-    if scale_const is not None:
+    if mode == "none":
+        s = None
+    elif scale_const is not None:
         s = np.full(sshape, scale_const, dtype=np.float64)
     else:
         s = r["scale"].uniform(scale_range[0], scale_range[1], size=sshape)
-    if offset and wdt != "fp8":
+    if offset and wdt != "fp8" and mode != "none":
         if offset_const is not None:
             o = np.full(sshape, offset_const, dtype=np.float64)
         elif fractional_offset:
@@ -209,7 +221,7 @@ def make_wqmm_case(*, name="case", x1_shape=(16, 256), n=128, act="bf16", wdt="i
     else:
         o = None
 
-    scale_bits = act_bits(s, act)
+    scale_bits = None if s is None else act_bits(s, act)
     off_bits = None if o is None else act_bits(o, act)
     if mode == "group" and scale_transposed:
         scale_bits = np.ascontiguousarray(scale_bits.T)
@@ -252,19 +264,26 @@ def make_qmm_case(*, name="qcase", x1_shape=(32, 64), n=128, out="bf16", bias=Tr
                    pertoken_scale=pt, x3=x3a, seed=seed)
 
 
-# --------------------------------------------------------------------------- the five workloads
+# --------------------------------------------------------------------------- the named workloads
+# The first five are the benchmark configurations of the operator's headline
+# comparison; the rest widen it: fp8-e4m3 weights (per-channel only, no
+# offset), a medium-m point, and the non-quantised scenario at the headline's
+# size.
 WORKLOADS = {
     "tiny_w8a16_perchannel_f16": "x1 f16 (16,256); x2 i8 (256,128); per-channel scale/offset; bias; no x3",
     "w8a16_pertensor_bf16_2048x4096x4096": "x1 bf16 (2048,4096); x2 i8 (4096,4096); scale=0.01 offset=3; bias; x3",
     "w4a16_g128_bf16_4096x4096x4096": "x1 bf16 (4096,4096); x2 i4 (4096,4096); g=128 scale/offset; no bias/x3",
     "decode_w4a16_g64_bf16_1x16x8192x28672": "x1 bf16 (1,16,8192); x2 i4 (8192,28672); g=64; bias",
     "w8a8_pertoken_4x2048x8192x1024": "x1 i8 (4,2048,8192); x2 i8 (8192,1024); bias i32; bf16 dq; pertoken; x3",
+    "fp8_perchannel_bf16_4096x4096x4096": "x1 bf16 (4096,4096); x2 fp8-e4m3 (4096,4096); per-channel scale; no offset",
+    "w4a16_g128_bf16_256x4096x4096": "x1 bf16 (256,4096); x2 i4 (4096,4096); g=128 scale/offset; no bias/x3",
+    "nonquant_bf16_4096x4096x4096": "x1 bf16 (4096,4096); x2 bf16 (4096,4096); no antiquant; no bias/x3",
 }
 WORKLOAD_NAMES = list(WORKLOADS)
 
 
 def workload(name: str):
-    """Build one of the five named workloads (seed = its index in WORKLOAD_NAMES)."""
+    """Build one of the named workloads (seed = its index in WORKLOAD_NAMES)."""
     i = WORKLOAD_NAMES.index(name)
     if i == 0:
         return make_wqmm_case(name=name, x1_shape=(16, 256), n=128, act="f16", wdt="i8", mode="channel",
@@ -283,4 +302,14 @@ def workload(name: str):
     if i == 4:
         return make_qmm_case(name=name, x1_shape=(4, 2048, 8192), n=1024, out="bf16", bias=True, x3=True,
                              pertoken=True, seed=4)
+    if i == 5:
+        return make_wqmm_case(name=name, x1_shape=(4096, 4096), n=4096, act="bf16", wdt="fp8", mode="channel",
+                              scale_range=(0.001, 0.02), offset=False, bias=False, x3=False, seed=5)
+    if i == 6:
+        return make_wqmm_case(name=name, x1_shape=(256, 4096), n=4096, act="bf16", wdt="i4", mode="group",
+                              group_size=128, scale_range=(0.005, 0.05), offset_range=(-4, 4),
+                              bias=False, x3=False, seed=6)
+    if i == 7:
+        return make_wqmm_case(name=name, x1_shape=(4096, 4096), n=4096, act="bf16", wdt="bf16",
+                              bias=False, x3=False, seed=7)
     raise KeyError(name)
