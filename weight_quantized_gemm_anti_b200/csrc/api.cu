@@ -872,9 +872,8 @@ wqmm_status run_wqmm(void* ws, wqmm_executor* ex, cudaStream_t s) {
   }
   CUtensorMap tmap;
   if (!ex->smallm) {  // the small-m kernel reads x1 with plain 16-byte copies
-    wqmm_status st = make_tmap(&tmap, ex->x1,
-                               bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ex->m,
-                               ex->k, kWqKTile, ex->pair ? ex->bn / 2 : ex->bn);
+    const CUtensorMapDataType dt = bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    wqmm_status st = make_tmap(&tmap, ex->x1, dt, 2, ex->m, ex->k, kWqKTile, ex->pair ? ex->bn / 2 : ex->bn);
     if (st) return st;
   }
   WqParams p{};

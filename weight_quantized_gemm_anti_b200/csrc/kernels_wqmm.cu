@@ -436,6 +436,7 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR, SPG>::kThreads, 1)
     // in turn
     constexpr bool kPrefetch = C::kThreads <= 512;
     float* wst = reinterpret_cast<float*>(s_stage) + quad * (kER * kEP);
+    const bool addends = p.bias != nullptr || p.x3 != nullptr;  // uniform: bias or x3 to add
     uint32_t j = 0;
     while (walk.next(p, it)) {
       const int ab = j % C::kNAcc;
@@ -561,11 +562,16 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR, SPG>::kThreads, 1)
             const float y[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
             const uint32_t xw[4] = {xv[ps].x, xv[ps].y, xv[ps].z, xv[ps].w};
             uint32_t o[4];
+            if (addends) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float a = y[2 * i] + bias8[2 * i] + act_f32(static_cast<uint16_t>(xw[i] & 0xFFFFu), BF16);
-              const float b = y[2 * i + 1] + bias8[2 * i + 1] + act_f32(static_cast<uint16_t>(xw[i] >> 16), BF16);
-              o[i] = pack2<BF16>(a, b);
+              for (int i = 0; i < 4; ++i) {
+                const float a = y[2 * i] + bias8[2 * i] + act_f32(static_cast<uint16_t>(xw[i] & 0xFFFFu), BF16);
+                const float b = y[2 * i + 1] + bias8[2 * i + 1] + act_f32(static_cast<uint16_t>(xw[i] >> 16), BF16);
+                o[i] = pack2<BF16>(a, b);
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) o[i] = pack2<BF16>(y[2 * i], y[2 * i + 1]);
             }
             *reinterpret_cast<uint4*>(p.out + mm * p.n + nn8) = make_uint4(o[0], o[1], o[2], o[3]);
           }
@@ -837,7 +843,7 @@ cudaError_t launch_spg(const CUtensorMap& tmap, const WqParams& p, int grid, cud
 
 template <int BN, bool PAIR, int WK, bool BF16>
 cudaError_t launch_mode(const CUtensorMap& tmap, const WqParams& p, int grid, cudaStream_t s) {
-  if constexpr (BN >= 128 && !PAIR && WK != kWH) {  // a 16-bit step fills a whole weight stage
+  if constexpr (BN >= 128 && WK != kWH) {  // a 16-bit step fills a whole weight stage
     if (p.kt_total % 2 == 0 && (!p.stream_k || p.sk_unit == 2))
       return launch_spg<BN, PAIR, WK, BF16, 2>(tmap, p, grid, s);
   }
