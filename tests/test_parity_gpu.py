@@ -157,6 +157,63 @@ def test_pack_kernel_16bit_layout():
     assert np.array_equal(got, want)
 
 
+# ---------------------------------------------------------------- row-parallel shards
+# The operator's tensor-parallel form splits x1 and x2 along k; each rank runs
+# the GEMM on its shard (bias and x3 included) and the AllReduce sums the
+# outputs.  Here every rank's part runs on this one GPU through the package's
+# shard helpers and matmul_all_reduce (no process group: the AllReduce is the
+# identity); the outputs are summed as a sum AllReduce would, and the sum is
+# held to the sum of the ranks' exact results.
+ROWPAR = [
+    ("rp_i4_g128_bf16", dict(x1_shape=(40, 1024), n=256, act="bf16", wdt="i4", mode="group", group_size=128,
+                             scale_range=(0.005, 0.05), offset_range=(-4, 4), seed=51), True),
+    ("rp_i4_g64_f16_transposed", dict(x1_shape=(24, 512), n=128, act="f16", wdt="i4", mode="group", group_size=64,
+                                      x2_transposed=True, scale_transposed=True, seed=52), True),
+    ("rp_i8_chan_bf16_m300", dict(x1_shape=(300, 640), n=192, act="bf16", wdt="i8", mode="channel", seed=53), False),
+    ("rp_fp8_chan_bf16", dict(x1_shape=(64, 512), n=128, act="bf16", wdt="fp8", mode="channel", offset=False,
+                              seed=55), False),
+    ("rp_nonquant_bf16", dict(x1_shape=(16, 512), n=128, act="bf16", wdt="bf16", seed=54), False),
+]
+
+
+@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("spec", ROWPAR, ids=[s[0] for s in ROWPAR])
+def test_row_parallel_shards_sum_to_the_operator(spec, world):
+    from rowparallel_cases import local_oracle, shard_case
+    from weight_quantized_gemm_anti_b200 import allreduce as AR
+    name, kw, int4 = spec
+    case = WL.make_wqmm_case(name=name, **kw)
+    adt = torch.bfloat16 if case.act == "bf16" else torch.float16
+    wcode = {"i8": W.DT_I8, "fp8": W.DT_FP8E4M3, "bf16": W.DT_BF16, "f16": W.DT_F16}.get(case.wdt)
+    dev = lambda t: None if t is None else t.cuda()
+    bias = None if case.bias is None else torch.from_numpy(case.bias.view(np.int16)).cuda().view(adt)
+    x3 = None if case.x3 is None else torch.from_numpy(case.x3.view(np.int16)).cuda().view(adt).reshape(case.out_shape)
+    total = np.zeros((case.m, case.n))
+    want = np.zeros((case.m, case.n))
+    bound = 0.0
+    for r in range(world):
+        k0, k1, x1, x2, sc, of = shard_case(case, r, world, int4)
+        x1 = x1.cuda().view(adt)
+        buf, x2d = AR.pack_shard(x2.cuda(), k1 - k0, case.n, int4=int4, transposed=case.x2_transposed, dtype=wcode)
+        sc, of = dev(sc), dev(of)
+        sc = None if sc is None else sc.view(adt)
+        of = None if of is None else of.view(adt)
+        if case.mode == "group" and case.scale_transposed:
+            sc, of = sc.t(), (None if of is None else of.t())
+        elif case.mode != "group" and sc is not None:
+            sc = sc.reshape(case.scale_shape)
+            of = None if of is None else of.reshape(case.scale_shape)
+        out = AR.matmul_all_reduce(x1, x2d, sc, of, bias, x3, case.group_size)
+        torch.cuda.synchronize()
+        no_device_error()
+        total += dec(gpu_bits(out), case.act)
+        ye = local_oracle(case, r, world, int4)
+        want += ye
+        bound += np.abs(ye).max()
+    err = np.abs(total - want).max() / bound
+    assert err <= TOL[case.act], f"{name} x{world}: {err:.3e}"
+
+
 # ---------------------------------------------------------------- small m (m <= 32)
 # The small-m kernel: dequantisation groups that issue their own MMAs, x1
 # fetched per turn by the groups, per-group scale/offset rows staged with the

@@ -263,6 +263,14 @@ def pack_weight(x2_desc: WqmmTensor, for_int8_gemm: bool = False, stream=None):
     return buf, desc(data=buf.data_ptr(), dtype=x2_desc.dtype, shape=(k, n), fmt=FORMAT_PACKED)
 
 
+def _keep_until_done(t, stream) -> None:
+    """A temporary used by work enqueued on `stream` stays allocated until that
+    work is done (the caching allocator reuses freed blocks only in the order
+    of the stream they are recorded on)."""
+    if t is not None and stream is not None and hasattr(stream, "cuda_stream"):
+        t.record_stream(stream)
+
+
 def _workspace(nbytes: int, device):
     import torch
     if nbytes == 0:
@@ -278,12 +286,14 @@ def weight_quant_matmul(x1, x2_desc: WqmmTensor, antiquant_scale, antiquant_offs
     if out is None:
         out = torch.empty(tuple(x1.shape[:-1]) + (x2_desc.shape[1],), dtype=x1.dtype, device=x1.device)
     st, ws_size, ex = wqmm_get_workspace_size(
-        desc(x1), x2_desc, None if bias is None else desc(bias), desc(antiquant_scale),
+        desc(x1), x2_desc, None if bias is None else desc(bias),
+        None if antiquant_scale is None else desc(antiquant_scale),
         None if antiquant_offset is None else desc(antiquant_offset), None if x3 is None else desc(x3), None, "sum",
         0, 1, antiquant_group_size, desc(out))
     check(st)
     ws, ws_ptr = _workspace(ws_size, x1.device)
     check(wqmm_run(ws_ptr, ws_size, ex, stream))
+    _keep_until_done(ws, stream)
     return out
 
 
@@ -305,4 +315,5 @@ def quant_matmul(x1, x2_desc: WqmmTensor, dequant_scale, pertoken_scale=None, bi
             check(rc)
     ws, ws_ptr = _workspace(ws_size, x1.device)
     check(qmm_run(ws_ptr, ws_size, ex, stream))
+    _keep_until_done(ws, stream)
     return out
