@@ -441,7 +441,8 @@ __global__ void __launch_bounds__(Cfg<BN, DG, WK, PAIR, SPG>::kThreads, 1)
     while (walk.next(p, it)) {
       const int ab = j % C::kNAcc;
       const bool ready =
-          mbar_wait_sleep(&bar_accfull[ab], (j / C::kNAcc) & 1, abort_flag, p.err, kDevTimeoutEpilogue, 64, 512);
+          // short sleeps: the drain of a finished tile should start promptly
+          mbar_wait_sleep(&bar_accfull[ab], (j / C::kNAcc) & 1, abort_flag, p.err, kDevTimeoutEpilogue, 32, 128);
       // one decision for all four warps: they meet at named barriers below
       if (!named_bar_and(1, 128, ready && !*abort_flag)) break;
       tc_fence_after();
