@@ -84,6 +84,8 @@ def wqmm_schedule(m: int, n: int, k: int, sms: int, nonquant: bool = False) -> d
     16-bit weight of the x1 dtype, which always runs on the general kernel."""
     bn = 16 if m <= 16 else 32 if m <= 32 else 64 if m <= 64 else 128 if m <= 128 else 256
     num_nb = -(-n // 128)
+    if 256 < m <= 512 and -(-m // 256) * num_nb < sms and -(-m // 128) * num_nb <= sms:
+        bn = 128  # the 128-row split is cheaper than the 256-row one here
     kt = -(-k // 64)
     tiles = -(-m // bn) * num_nb
     out = {"bn": bn, "stream_k": False, "inline": False, "partial_bytes": 0, "flag_bytes": 0,

@@ -266,6 +266,8 @@ def test_pack_size_queries():
     (16, 4096, 256),       # 2 tiles over many CTAs: fix-up kernel
     (300, 512, 256),       # wide tiles, fewer than the CTAs: two-step units
     (200, 448, 384),       # odd k-step count
+    (384, 4096, 4096),     # medium m: 128-row tiles split over the SMs
+    (512, 1024, 8192),     # medium m with enough 128-row tiles for whole waves: 256 rows
 ])
 @pytest.mark.parametrize("nonquant", [False, True], ids=["int4", "nonquant"])
 def test_schedule_mirror_matches_library_workspace(m, k, n, nonquant):

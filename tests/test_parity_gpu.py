@@ -106,6 +106,7 @@ SMALL = [
     ("i8_splitk_m5", (5, 2048), 128, "f16", "i8", "channel", 0, {}),
     ("i4_m64_bn64", (64, 512), 256, "bf16", "i4", "group", 64, {}),
     ("i4_m20_bn32", (20, 512), 512, "bf16", "i4", "group", 32, {}),
+    ("i4_g128_bf16_m384_split128", (384, 512), 256, "bf16", "i4", "group", 128, {}),
 ]
 
 

@@ -485,6 +485,15 @@ extern "C" wqmm_status wqmm_get_workspace_size(const wqmm_tensor* x1, const wqmm
     // m tile: the smallest supported width that covers m; larger m uses 256,
     // the widest MMA (the most MMA work per dequantised weight step)
     ex->bn = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <= 128 ? 128 : 256;
+    {
+      // 256 < m <= 512 with fewer tiles than SMs at both 256 and 128 rows: every
+      // tile is split over the SMs either way, and the 128-row split is cheaper
+      // than the 256-row one (measured on B200, W4A16 g128, k = n = 4096:
+      // m = 384 43.0 vs 55.2 us, m = 512 47.1 vs 55.3 us)
+      const int64_t nb = (n + kWqNBlock - 1) / kWqNBlock;
+      const int64_t sl = sm_count();
+      if (m > 256 && m <= 512 && ((m + 255) / 256) * nb < sl && ((m + 127) / 128) * nb <= sl) ex->bn = 128;
+    }
     if (const char* env = std::getenv("WQMM_BN")) {  // tuning override
       const int v = std::atoi(env);
       if (v == 16 || v == 32 || v == 64 || v == 128 || v == 192 || v == 256) ex->bn = v;
