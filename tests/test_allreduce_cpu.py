@@ -131,3 +131,10 @@ def test_int4_shards_hold_the_same_values():
             s = AR.shard_weight(full, k0, k1, int4=True, transposed=transposed).numpy()
             got = unpack(s, case.n, k1 - k0).T if transposed else unpack(s, k1 - k0, case.n)
             assert np.array_equal(got, ref[k0:k1])
+
+
+def test_matmul_all_reduce_takes_a_torch_stream_only():
+    # the AllReduce is ordered on the stream the GEMM ran on, which needs a
+    # torch.cuda.Stream (a raw handle cannot be waited on by the process group)
+    with pytest.raises(TypeError):
+        AR.matmul_all_reduce(None, None, stream=12345)

@@ -14,8 +14,9 @@ output tensor's dtype.
 
 One process per GPU: each rank runs this library's GEMM on its shard, then
 torch.distributed.all_reduce(SUM) on the output (ncclAllReduce with the NCCL
-backend, on the process group's own stream ordered after the GEMM).  At
-world size 1 the AllReduce is the identity and nothing is launched for it.
+backend, on the process group's own stream, which waits for the stream the
+GEMM was enqueued on).  At world size 1 the AllReduce is the identity and
+nothing is launched for it.
 
 Shards: a rank's k range starts on a multiple of lcm(64, G) (G = the
 per-group size, or 1): whole 64-wide k steps of the packed weight and whole
@@ -78,12 +79,19 @@ def shard_group_rows(t, k0: int, k1: int, group_size: int, *, transposed: bool =
     return (t[:, g0:g1] if transposed else t[g0:g1]).contiguous()
 
 
-def all_reduce_output(out, group=None):
+def all_reduce_output(out, group=None, stream=None):
     """Sum `out` over the ranks of `group` in place (the operator's AllReduce,
-    reduceOp "sum"); the identity when there is one rank or no process group."""
+    reduceOp "sum"); the identity when there is one rank or no process group.
+    The collective is ordered after the work already enqueued on `stream` (a
+    torch.cuda.Stream; None: the current stream)."""
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
-        dist.all_reduce(out, op=dist.ReduceOp.SUM, group=group)
+        if stream is not None and hasattr(stream, "cuda_stream"):
+            import torch
+            with torch.cuda.stream(stream):
+                dist.all_reduce(out, op=dist.ReduceOp.SUM, group=group)
+        else:
+            dist.all_reduce(out, op=dist.ReduceOp.SUM, group=group)
     return out
 
 
@@ -106,7 +114,11 @@ def matmul_all_reduce(x1, x2_desc, antiquant_scale=None, antiquant_offset=None, 
     shard (x1: this rank's k columns; x2_desc: its k rows, e.g. from
     pack_shard; scale/offset: its group rows, or the full per-channel /
     per-tensor tensors), then the AllReduce(sum) of the output over `group`.
-    antiquant_scale None: the non-quantised scenario (x2 of the x1 dtype)."""
+    antiquant_scale None: the non-quantised scenario (x2 of the x1 dtype).
+    `stream`: a torch.cuda.Stream (or None for the current stream) that both the
+    GEMM and the AllReduce are ordered on."""
+    if stream is not None and not hasattr(stream, "cuda_stream"):
+        raise TypeError("stream must be a torch.cuda.Stream or None")
     out = weight_quant_matmul(x1, x2_desc, antiquant_scale, antiquant_offset, bias, x3, antiquant_group_size, out,
                               stream)
-    return all_reduce_output(out, group)
+    return all_reduce_output(out, group, stream)
