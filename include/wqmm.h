@@ -10,7 +10,9 @@
  *             output = dequantScale * pertokenScale * (x1_int8 @ x2_int8 + bias_int32) + x3
  *
  * The AllReduce of both operators is the identity for one rank and is not
- * performed here.  Every call follows the two-phase convention of those pages
+ * performed by these entry points; across ranks (row-parallel, x1 and x2
+ * split along k) the Python package runs the GEMM per rank and sums the
+ * outputs with an NCCL all-reduce (weight_quantized_gemm_anti_b200.allreduce).  Every call follows the two-phase convention of those pages
  * ("两段式接口与函数原型"; "Function Prototype"): phase 1 validates the
  * arguments, plans the launch and reports the device workspace it needs; the
  * caller allocates that workspace (only when the size is > 0) and calls phase
