@@ -25,6 +25,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import subprocess
 import sys
 import tempfile
@@ -44,11 +45,20 @@ KERNEL_SOURCES = ["weight_quantized_gemm_anti_b200/csrc/kernels_wqmm.cu",
                   "weight_quantized_gemm_anti_b200/csrc/kernels_aux.cu"]
 
 
+def _code_only(text: str) -> str:
+    """C/C++/CUDA source without comments and with whitespace collapsed, so that
+    the hash follows the code, not its documentation."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash() -> str:
+    """Identifies the kernel code a profile was taken on (comments ignored)."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, f), encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -19,15 +19,24 @@
 //               TMEM (two buffers when they fit, so the epilogue of one tile
 //               overlaps the main loop of the next); stages are released with
 //               tcgen05.commit;
-//   warps 2..5  epilogue (one per TMEM lane quadrant): tcgen05.ld of the
-//               accumulator, fp32 scale / + bias / + x3, one rounding, store --
-//               or an fp32 partial tile in stream-K mode;
+//   warps 2..5  epilogue (one per TMEM lane quadrant, each on its own):
+//               tcgen05.ld of the accumulator 16 columns at a time, fp32 scale,
+//               staging of the warp's 32 columns, + bias / + x3, one rounding,
+//               16-byte stores -- or an fp32 partial tile in stream-K mode;
 //   warps 7..   DG dequantisation groups of four warps (one per lane
-//               quadrant; thread = weight column).  Group g takes the k steps
-//               g, g+DG, ...: loads its column's per-group scale/offset from
-//               L2 one step ahead, unpacks its column's 64 weights, dequantises them
-//               in registers and tcgen05.st's them into one of its own TMEM A
-//               stages, so DG k steps are dequantised concurrently.
+//               quadrant; thread = weight column).  Group g takes turns of SPG
+//               consecutive k steps (steps g*SPG .. g*SPG+SPG-1 mod DG*SPG):
+//               loads its column's per-group scale/offset from L2 one turn
+//               ahead, unpacks its column's weights, dequantises them in
+//               registers and tcgen05.st's them into its own TMEM A stages, so
+//               DG turns are dequantised concurrently (DG = 2, SPG = 2 for
+//               wide tiles with an even k-step count, single CTAs and CTA
+//               pairs alike; DG = 4, SPG = 1 otherwise).  16-bit weights (the
+//               non-quantised scenario) are stored to the A stages as they are.
+//
+// CTA pairs (256-row m tiles, int4 by default): clusters of two CTAs share
+// each MMA (cta_group::2, M = 256 weight columns); each CTA holds half of the
+// x1 slab and its own 128 weight columns, and only the even CTA issues.
 //
 // Work is whole output tiles dealt round-robin to the CTAs, optionally
 // followed by "stream-K" tiles whose k steps are split evenly over the CTAs
