@@ -299,6 +299,23 @@ def workload_roofline(prob, peaks, int8_peak):
     return bound, peaks["hbm_gbs"], "GB/s", "HBM copy"
 
 
+def algorithmic_bytes(case) -> float:
+    """Each input read once plus the output written once (int4 = 0.5 B)."""
+    c = case
+    if not hasattr(c, "wdt"):
+        b = c.m * c.k + c.k * c.n + c.m * c.n * 2
+        b += 0 if c.bias is None else 4 * c.n
+        b += c.dequant_scale.nbytes + (0 if c.pertoken_scale is None else 4 * c.m)
+        b += 0 if c.x3 is None else 2 * c.m * c.n
+        return b
+    wbytes = {"i4": 0.5, "i8": 1.0, "fp8": 1.0, "f16": 2.0, "bf16": 2.0}[c.wdt]
+    b = c.m * c.k * 2 + c.k * c.n * wbytes + c.m * c.n * 2
+    b += (0 if c.scale is None else c.scale.nbytes) + (0 if c.offset is None else c.offset.nbytes)
+    b += 0 if c.bias is None else 2 * c.n
+    b += 0 if c.x3 is None else 2 * c.m * c.n
+    return b
+
+
 # ------------------------------------------------------------------ GPU arm
 class Problem:
     """One workload resident on the device, with prebuilt ABI descriptors."""
@@ -320,7 +337,7 @@ class Problem:
         torch.cuda.synchronize()
         c = self.case
         self.flops = 2.0 * c.m * c.n * c.k
-        self.bytes = self._algorithmic_bytes()
+        self.bytes = algorithmic_bytes(self.case)
         d = self.dev
         D = W.desc
         if self.int8:
@@ -334,22 +351,6 @@ class Problem:
         W.wqmm_executor_destroy(ex)
         self.ws_size = ws
         self.ws = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
-
-    def _algorithmic_bytes(self):
-        """Each input read once plus the output written once (int4 = 0.5 B)."""
-        c = self.case
-        if self.int8:
-            b = c.m * c.k + c.k * c.n + c.m * c.n * 2
-            b += 0 if c.bias is None else 4 * c.n
-            b += c.dequant_scale.nbytes + (0 if c.pertoken_scale is None else 4 * c.m)
-            b += 0 if c.x3 is None else 2 * c.m * c.n
-            return b
-        wbytes = {"i4": 0.5, "i8": 1.0, "fp8": 1.0, "f16": 2.0, "bf16": 2.0}[c.wdt]
-        b = c.m * c.k * 2 + c.k * c.n * wbytes + c.m * c.n * 2
-        b += (0 if c.scale is None else c.scale.nbytes) + (0 if c.offset is None else c.offset.nbytes)
-        b += 0 if c.bias is None else 2 * c.n
-        b += 0 if c.x3 is None else 2 * c.m * c.n
-        return b
 
     def phase1(self):
         if self.int8:
