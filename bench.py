@@ -523,7 +523,9 @@ def gpu_arm(args):
             if nm == args.config:
                 continue
             p2 = Problem(nm, f"cuda:{local}")
-            tt, _ = time_device(p2, max(args.extra_steps, 50), 3, flush_bytes)
+            # launch-latency-sized problems: a larger sample for a stable median
+            nsteps = 1000 if p2.flops < 1e8 else max(args.extra_steps, 50)
+            tt, _ = time_device(p2, nsteps, 3, flush_bytes)
             tt.sort()
             ms = tt[len(tt) // 2]  # median step
             bound, peak, unit, src = workload_roofline(p2, peaks, int8_peak)
