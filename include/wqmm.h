@@ -107,8 +107,9 @@ typedef struct CUstream_st* wqmm_stream; /* a cudaStream_t; NULL = the legacy de
  *                    its dtype then equals x1's): output = x1 @ x2 + bias + x3, with
  *                    antiquant_scale and antiquant_offset NULL and G = 0.
  *  bias              optional, (n), dtype of x1.
- *  antiquant_scale   required for int8 / int4 / fp8 weights (NULL otherwise:
- *                    WQMM_ERR_PARAM_NULLPTR), dtype of x1: per-tensor (1); per-channel (n) or (1, n);
+ *  antiquant_scale   required for int8 / int4 / fp8 weights (a NULL scale there is
+ *                    WQMM_ERR_PARAM_NULLPTR), NULL for f16 / bf16 weights (a scale there is
+ *                    WQMM_ERR_PARAM_INVALID); dtype of x1: per-tensor (1); per-channel (n) or (1, n);
  *                    per-group (ceil(k / G), n) -- contiguous, or transposed (strides
  *                    (1, ceil(k/G))) exactly when x2 is transposed ("约束说明").
  *  antiquant_offset  optional, same shape, dtype and strides as the scale; ADDED to the
