@@ -5,6 +5,8 @@ and workspace checks fail with a status and launch nothing."""
 import os
 
 import pytest
+from hypothesis import given, settings
+from hypothesis import strategies as st
 
 import weight_quantized_gemm_anti_b200 as W
 
@@ -287,3 +289,19 @@ def test_schedule_mirror_matches_library_workspace(m, k, n, nonquant):
     s = bench.wqmm_schedule(m, n, k, sms, nonquant=nonquant)
     rnd = lambda b: -(-b // 256) * 256
     assert ws == rnd(s["partial_bytes"]) + rnd(s["flag_bytes"]), (s, ws)
+
+
+@settings(max_examples=80, deadline=None, derandomize=True)
+@given(m=st.integers(1, 3000), k_steps=st.integers(1, 160), n_blocks=st.integers(1, 400), nonquant=st.booleans())
+def test_schedule_mirror_random_shapes(m, k_steps, n_blocks, nonquant):
+    # the benchmark's restatement of the planner agrees with phase 1's
+    # workspace (split-tile partials and flags) over random shapes
+    import bench
+    k, n = 64 * k_steps, 64 * n_blocks
+    dt = W.DT_BF16 if nonquant else W.DT_I4
+    st_, ws = wq(x1=((m, k), W.DT_BF16), x2=((k, n), dt), scale=None if nonquant else ((n,), None),
+                 x2_fmt=W.FORMAT_PACKED)
+    assert st_ == W.SUCCESS
+    s = bench.wqmm_schedule(m, n, k, 148, nonquant=nonquant)
+    rnd = lambda b: -(-b // 256) * 256
+    assert ws == rnd(s["partial_bytes"]) + rnd(s["flag_bytes"]), (m, k, n, nonquant, s, ws)
