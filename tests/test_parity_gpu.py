@@ -1,10 +1,11 @@
 """GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
 same seeded inputs.
 
-Tolerance (stated by the task for this operator): max|gpu - oracle| / max|oracle|
-<= 4e-3 for bf16 outputs and <= 1e-3 for fp16 outputs, where `oracle` is the
-exact (fp64, pre-rounding) result; the raw int32 accumulator of the int8 path
-is compared bit for bit.  Small cases span several tiles plus ragged tails in
+Tolerance: max|gpu - oracle| / max|oracle| <= 4e-3 for bf16 outputs and
+<= 1e-3 for fp16 outputs, where `oracle` is the exact (fp64, pre-rounding)
+result -- the budget of one rounding of each dequantised weight to the MMA
+operand type plus one rounding of the output; the raw int32 accumulator of the
+int8 path is compared bit for bit.  Small cases span several tiles plus ragged tails in
 m, n and k and cover every mode, weight type, activation type and layout;
 full-size workloads are checked on sampled outputs the oracle evaluates one by
 one.
