@@ -17,6 +17,8 @@ import socket
 
 import numpy as np
 import pytest
+from hypothesis import given, settings
+from hypothesis import strategies as st
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
@@ -138,3 +140,25 @@ def test_matmul_all_reduce_takes_a_torch_stream_only():
     # torch.cuda.Stream (a raw handle cannot be waited on by the process group)
     with pytest.raises(TypeError):
         AR.matmul_all_reduce(None, None, stream=12345)
+
+
+@settings(max_examples=200, deadline=None, derandomize=True)
+@given(k_units=st.integers(1, 1024), world=st.integers(1, 8), g=st.sampled_from([0, 32, 64, 96, 128, 192, 256]),
+       tail=st.integers(0, 63))
+def test_k_ranges_properties(k_units, world, g, tail):
+    # any k (a ragged tail included) and world: contiguous cover of [0, k),
+    # starts on whole 64-wide steps and whole groups, balanced to one unit,
+    # or a refusal when there are fewer units than ranks
+    unit = AR.k_shard_unit(g)
+    k = 64 * k_units + (tail // 32) * 32
+    units = -(-k // unit)
+    if units < world:
+        with pytest.raises(ValueError):
+            AR.k_ranges(k, world, g)
+        return
+    r = AR.k_ranges(k, world, g)
+    assert r[0][0] == 0 and r[-1][1] == k and len(r) == world
+    assert all(b == c for (_, b), (c, _) in zip(r, r[1:]))
+    assert all(a % unit == 0 and b > a for a, b in r)
+    sizes = [-(-(b - a) // unit) for a, b in r]
+    assert max(sizes) - min(sizes) <= 1 and sum(sizes) == units

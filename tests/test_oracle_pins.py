@@ -273,6 +273,21 @@ def test_qmm_matches_exact_integer_brute_force():
             assert float(dec_bf16(yr[i, j])) == float(rne_act(e, "bf16"))
 
 
+@settings(max_examples=30, deadline=None, derandomize=True)
+@given(m=st.integers(1, 6), k=st.integers(1, 80), n=st.integers(1, 6), out=st.sampled_from(["bf16", "f16"]),
+       pertoken=st.booleans(), dq_per_tensor=st.booleans(), bias=st.booleans(), seed=st.integers(0, 10_000))
+def test_qmm_random_shapes_exact_accumulator(m, k, n, out, pertoken, dq_per_tensor, bias, seed):
+    # the int8 path's accumulator is the exact integer product plus bias (no
+    # wrap at these sizes), over random shapes and options
+    case = W.make_qmm_case(x1_shape=(m, k), n=n, out=out, bias=bias, x3=True, pertoken=pertoken,
+                           dq_per_tensor=dq_per_tensor, seed=seed)
+    acc, ye, _ = oracle.qmm(case)
+    want = case.x1.astype(np.int64) @ case.x2.astype(np.int64)
+    if case.bias is not None:
+        want = want + case.bias.astype(np.int64)[None, :]
+    assert np.array_equal(acc.astype(np.int64), want)
+
+
 def test_qmm_int32_wraps_like_a_32bit_accumulator():
     case = W.make_qmm_case(x1_shape=(2, 32), n=3, out="bf16", seed=9, pertoken=False, x3=False)
     case.x1[:] = 127
